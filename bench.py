@@ -1,0 +1,360 @@
+"""Benchmark of the quantized-Linear hot path on B200.
+
+Workload (one step): the decode GEMV sweep at M = 1 -- the four distinct
+projection shapes of a Qwen2.5-VL-3B-class block (K x N = 2048x2048 q/o,
+2048x256 k/v, 2048x11008 gate/up, 11008x2048 down) in three packs each
+(INT4 group 128, INT4 group 64, NVFP4): 12 quantized Linear calls on seeded
+synthetic bf16 weights ~N(0, 0.02) with 0.5% outlier input channels x20 and
+activations ~N(0, 1).  Metric: algorithmic bytes (packed weights + scales +
+zero points + activations + outputs) per second.  Weights rotate over enough
+copies that every step reads them from HBM, not L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (under torchrun) every rank runs the same per-GPU sweep on its own
+weights: independent problems, no collective on the data path (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 linear GB/s (M=1) and TFLOP/s (M≥512) as % of B200 roofline"
+WORKLOAD = ("decode GEMV sweep, M=1: K x N in {2048x2048, 2048x256, 2048x11008, 11008x2048} "
+            "x {INT4 g128, INT4 g64, NVFP4}, bf16 activations")
+FORMATS = (("int4", 128), ("int4", 64), ("nvfp4", 0))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), reasons=parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = set()
+        for r in rows:
+            for n, v in zip(names[1:], r["reasons"][1:]):
+                if v.lower().startswith("active"):
+                    seen.add(n)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(seen), "samples": len(rows)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+
+    import w4a16_gemm_wq_b200 as wq
+    from w4a16_gemm_wq_b200 import synth
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    wq.load()
+    peaks = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    # ---- build the rotating weight sets (each copy: 4 shapes x 3 packs)
+    def make_set(copy):
+        layers = []
+        for si, (K, N) in enumerate(synth.DECODE_SHAPES):
+            W = synth.weight(N, K, seed=synth.layer_seed(2, 100 * copy + si + 1000 * rank), device=dev)
+            for fmt, G in FORMATS:
+                p = wq.wq_quantize_nvfp4(W) if fmt == "nvfp4" else wq.wq_quantize_int4(W, G, 1)
+                layers.append((fmt, G, K, N, p))
+            del W
+        return layers
+
+    set_bytes = 0
+    first = make_set(0)
+    for fmt, G, K, N, p in first:
+        set_bytes += p.nbytes()
+    copies = max(2, -(-(2 * l2) // set_bytes) + 1)
+    sets = [first] + [make_set(c) for c in range(1, copies)]
+    torch.cuda.synchronize()
+
+    X = {K: synth.activations(1, K, seed=synth.layer_seed(2, K), device=dev) for K, _ in synth.DECODE_SHAPES}
+    Y = {N: torch.empty((1, N), dtype=torch.bfloat16, device=dev) for _, N in synth.DECODE_SHAPES}
+
+    def layer_bytes(fmt, G, K, N, p):
+        return p.nbytes() + 2 * K + 2 * N
+
+    step_bytes = sum(layer_bytes(*l) for l in first)
+
+    def linear(fmt, p, x, y):
+        if fmt == "nvfp4":
+            wq.wq_linear_nvfp4(x, p, out=y)
+        else:
+            wq.wq_linear_int4(x, p, out=y)
+
+    def step(i, events=None):
+        for j, (fmt, G, K, N, p) in enumerate(sets[i % len(sets)]):
+            if events is not None:
+                events[j][0].record()
+            linear(fmt, p, X[K], Y[N])
+            if events is not None:
+                events[j][1].record()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    nl = len(first)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nl)]
+          for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        start.record()
+        for i in range(args.steps):
+            step(args.warmup + i, ev[i])
+        stop.record()
+        torch.cuda.synchronize()
+    ms = start.elapsed_time(stop)
+    kernel_ms = sum(a.elapsed_time(b) for row in ev for a, b in row)
+    if pg:
+        t = torch.tensor([ms, kernel_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms, kernel_ms = t.tolist()
+
+    # per-shape breakdown (GB/s of each launch kind, averaged over steps)
+    detail = {}
+    for j, (fmt, G, K, N, p) in enumerate(first):
+        t_ms = sum(ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(args.steps)) / args.steps
+        key = f"{fmt}{'_g' + str(G) if G else ''}_{K}x{N}"
+        detail[key] = {"us": round(t_ms * 1e3, 2), "GB/s": round(layer_bytes(fmt, G, K, N, p) / (t_ms * 1e-3) / 1e9, 1)}
+
+    value = ws * step_bytes * args.steps / (ms * 1e-3) / 1e9
+    achieved = step_bytes * args.steps / (kernel_ms * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers (pinned), per step:
+    # H2D of the step's activations, the 12 linear calls, D2H of the outputs.
+    hx = {K: X[K].cpu().pin_memory() for K in X}
+    hy = {N: torch.empty((1, N), dtype=torch.bfloat16).pin_memory() for N in Y}
+    dx = {K: torch.empty_like(X[K]) for K in X}
+
+    def e2e_step(i):
+        for j, (fmt, G, K, N, p) in enumerate(sets[i % len(sets)]):
+            dx[K].copy_(hx[K], non_blocking=True)
+            linear(fmt, p, dx[K], Y[N])
+            hy[N].copy_(Y[N], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for i in range(args.steps):
+        e2e_step(args.warmup + i)
+    e2.record()
+    torch.cuda.synchronize()
+    ms2 = s2.elapsed_time(e2)
+    if pg:
+        t = torch.tensor([ms2], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms2 = t.item()
+    h2d = sum(2 * K for (_, _, K, _, _) in first)
+    d2h = sum(2 * N for (_, _, _, N, _) in first)
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "bytes_per_step": step_bytes,
+                   "l2_flush": f"inputs rotate over {copies} weight copies ({copies * set_bytes / 1e6:.0f} MB) "
+                               f"> 2x L2 ({l2 / 1e6:.0f} MB)",
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "kernel": "gemv_kernel", "achieved": round(achieved, 1),
+                     "peak": peaks["hbm"], "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
+                     "peak_source": peaks["source"], "traffic": None},
+        "e2e": {"value": round(ws * step_bytes * args.steps / (ms2 * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": nl * args.steps,
+        "detail": detail,
+    }
+    out["clocks"] = clk.summary()
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_sample_step(cache, frac_rows: int):
+    """Oracle on a bounded sample of one step: every 12 linear calls of the sweep
+    on 1/frac_rows of the output rows (dequantize those rows in fp64, fp64 dot)."""
+    import numpy as np
+
+    import oracle
+
+    nbytes = 0
+    for (fmt, G, K, N, pk, X) in cache:
+        rows = np.arange(0, N, frac_rows)
+        if fmt == "nvfp4":
+            wh = oracle.dequant_nvfp4(pk, rows=rows)
+            nbytes += len(rows) * (K // 2 + K // 16) + 2 * K + 2 * len(rows)
+        else:
+            wh = oracle.dequant_int4(pk, rows=rows)
+            nbytes += len(rows) * (K // 2 + 2 * (K // G) + 4 * (-(-(K // G) // 8))) + 2 * K + 2 * len(rows)
+        oracle.linear(X, wh)
+    return nbytes
+
+
+def oracle_cache():
+    import oracle
+    from w4a16_gemm_wq_b200 import synth
+
+    cache = []
+    for si, (K, N) in enumerate(synth.DECODE_SHAPES):
+        W = synth.weight(N, K, seed=synth.layer_seed(2, si + 1))
+        X = synth.activations(1, K, seed=synth.layer_seed(2, K))
+        for fmt, G in FORMATS:
+            pk = oracle.quantize_nvfp4(W) if fmt == "nvfp4" else oracle.quantize_int4(W, G)
+            cache.append((fmt, G, K, N, pk, X))
+    return cache
+
+
+def cpu_baseline(seconds: float = 10.0):
+    import oracle
+
+    cache = oracle_cache()
+    frac = 4
+    oracle_sample_step(cache, frac)  # warm
+    t0 = time.perf_counter()
+    nbytes, n = 0, 0
+    while time.perf_counter() - t0 < seconds:
+        nbytes += oracle_sample_step(cache, frac)
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} passes of the 12-call decode sweep on every {frac}th output row "
+                      f"(fp64 dequantize + fp64 dot), {dt:.1f} s"}
+
+
+def run_reference(args):
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return
+    import oracle
+
+    cache = oracle_cache()
+    frac = 16
+    for _ in range(args.warmup):
+        oracle_sample_step(cache, frac)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for _ in range(args.steps):
+        nbytes += oracle_sample_step(cache, frac)
+    dt = time.perf_counter() - t0
+    v = nbytes / dt / 1e9
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": ws,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": WORKLOAD, "sample": f"every {frac}th output row"},
+           "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                            "sample": f"each step: the 12-call decode sweep on every {frac}th output row"},
+           "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * wq.h -- C ABI of libwq, a B200 (sm_100a) library for group-wise 4-bit
+ * weight-only quantization of transformer Linear layers and for the
+ * quantized Linear Y = X * dequant(Wq)^T with bf16 activations.
+ *
+ * Method (page titles and sections):
+ *  - "Lance-Quant" (zingnex.cn), section "量化应用": AWQ-style grid search of
+ *    an activation-aware per-input-channel scale, group-wise INT4 packing,
+ *    and the NVFP4 pack (E2M1 codes with one FP8-E4M3 scale per 16
+ *    elements) for Blackwell tensor cores; section "当前局限": the quantized
+ *    Linear should run as a fused dequant GEMM, not a dequant-then-matmul.
+ *  - "quantization primer" (xingyuwang.me), section 2: asymmetric
+ *    q = round(x/s) + z, x_hat = (q - z) s with clipping; section 3:
+ *    per-group scales; section 4: W4A16 (4-bit weights, 16-bit
+ *    activations); section 12: FP8 E4M3 bit layout; section 13: a fused
+ *    kernel reads compressed weights and dequantizes inside the matmul.
+ *  - "OmniQuant" tutorial (cyqw.cn), section 2.1: scale and zero point;
+ *    section 2.2.2: the equivalence Y = (X s)(W / s); section 4.2: W4A4.
+ *
+ * Conventions for every entry point:
+ *  - Matrices are row-major.  W and Wq are [N, K] (N = out_features, row n
+ *    holds the K input-channel weights of output n); X is [M, K]; Y [M, N].
+ *  - bf16 and fp16 values travel as their 16-bit patterns (uint16_t).
+ *  - All data pointers are DEVICE pointers owned by the caller; the library
+ *    allocates no memory and keeps no state except one device error word
+ *    per loaded GPU (see wq_device_error).
+ *  - `stream` is a cudaStream_t (0 = legacy default stream).  Every call is
+ *    asynchronous on that stream; validation happens on the host before any
+ *    launch, so an error return means nothing was launched.
+ *  - Data pointers must be 16-byte aligned; K must be a multiple of 32.
+ *  - Status codes mirror the exit codes 0 / 1 / 2 of the "llm-quantize"
+ *    guide (blog.yoooo.fun): 0 ok, 1 argument validation failed, 2 runtime
+ *    (CUDA) failure; 3 = valid but unsupported parameters; 4 = a kernel's
+ *    bounded wait ran out (reported by wq_device_error).
+ *
+ * Packed INT4 format (the pages fix no layout; this library's choice):
+ *    qweight uint32 [N, K/8]   nibble j (bits 4j..4j+3) of word k/8 = code of k%8 == j
+ *    scales  fp16   [N, K/G]   one scale per group of G consecutive k
+ *    zeros   uint32 [N, ceil(K/G/8)]  nibble g%8 of word g/8 = zero point of
+ *                              group g; unused high nibbles of the last word are 0
+ *    asymmetric (zero_point=1): w_hat = (q - z) * scale
+ *    symmetric  (zero_point=0): w_hat = (q - 8) * scale, no zeros buffer
+ * Packed NVFP4 format:
+ *    codes   uint8 [N, K/2]    low nibble = element 2j, high nibble = 2j+1,
+ *                              E2M1 (1 sign, 2 exponent, 1 mantissa)
+ *    bscale  uint8 [N, K/16]   FP8 E4M3 block scale, one per 16 consecutive k
+ *    global_scale float [1]    per-tensor fp32 scale g
+ *    w_hat = e2m1(code) * e4m3(bscale) * g
+ */
+#ifndef WQ_H_
+#define WQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WQ_OK = 0,
+  WQ_ERR_ARG = 1,         /* null/misaligned pointer, bad size, too-small workspace */
+  WQ_ERR_CUDA = 2,        /* a CUDA launch or runtime call failed */
+  WQ_ERR_UNSUPPORTED = 3, /* bits != 4, group_size not in {64, 128}, ... */
+  WQ_ERR_TIMEOUT = 4      /* a device-side bounded wait gave up (see wq_device_error) */
+} wq_status;
+
+/* Linear formats for wq_linear_workspace_size. */
+enum { WQ_FMT_INT4 = 0, WQ_FMT_NVFP4 = 1 };
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* wq_status_string(int status);
+
+/* Message of the last error this thread saw inside the library ("" if none). */
+const char* wq_last_error(void);
+
+/* ---------------------------------------------------------------- sizes
+ * Host-only; no device work.  Byte counts of the packed buffers above. */
+int wq_int4_sizes(int64_t N, int64_t K, int group_size, size_t* qweight_bytes,
+                  size_t* scales_bytes, size_t* zeros_bytes);
+int wq_nvfp4_sizes(int64_t N, int64_t K, size_t* codes_bytes, size_t* bscale_bytes);
+
+/* Scratch bytes wq_linear_int4 / wq_linear_nvfp4 need for an [M, K] x [N, K]
+ * problem (format WQ_FMT_*, act_fp4 as in wq_linear_nvfp4).  0 means the call
+ * needs no workspace and accepts ws = NULL. */
+int wq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int format, int act_fp4,
+                             size_t* bytes);
+
+/* Scratch bytes awq_search_scale needs. */
+int awq_search_workspace_size(int64_t N, int64_t K, int64_t T, int n_alpha, int group_size,
+                              size_t* bytes);
+
+/* ---------------------------------------------------------------- stage 1: quantize + pack
+ * wq_quantize_int4 -- group-wise INT4 quantization ("quantization primer"
+ * sections 2-3; "Lance-Quant" section "量化应用": pack by group).
+ *   W        bf16 [N, K]
+ *   bits     must be 4
+ *   group_size 64 or 128 (K % group_size == 0)
+ *   zero_point 1 = asymmetric with per-group zero point, 0 = symmetric
+ *   scale_s  fp32 [K] AWQ per-input-channel scale, or NULL; when given the
+ *            library quantizes w' = W[n,k] * scale_s[k] (fp32 multiply)
+ *   qweight, scales, zeros: outputs in the packed INT4 format above; zeros
+ *            must be NULL when zero_point == 0 and non-NULL otherwise.
+ * Per group (all fp32, IEEE round-to-nearest-even, rint ties to even):
+ *   asymmetric: scale = fp16(clamp((max - min) / 15, 1e-5, 65504)),
+ *               z = clamp(rint(-min / scale), 0, 15),
+ *               q = clamp(rint(w' / scale) + z, 0, 15)
+ *   symmetric:  scale = fp16(clamp(max|w'| / 7, 1e-5, 65504)),
+ *               q = clamp(rint(w' / scale), -7, 7) + 8
+ * Results are bit-for-bit deterministic. */
+int wq_quantize_int4(const uint16_t* W, int64_t N, int64_t K, int bits, int group_size,
+                     int zero_point, const float* scale_s, uint32_t* qweight, uint16_t* scales,
+                     uint32_t* zeros, void* stream);
+
+/* wq_quantize_nvfp4 -- NVFP4 pack ("Lance-Quant" section "量化应用": E2M1 +
+ * FP8-E4M3 per 16 elements; "quantization primer" section 12: E4M3 layout).
+ *   W        bf16 [N, K] (K % 16 == 0; K % 32 == 0 as everywhere)
+ *   scale_s  fp32 [K] or NULL, as for INT4
+ *   codes, bscale, global_scale: outputs in the packed NVFP4 format above.
+ * g = amax|w'| / (6 * 448) (1 if all zero); per block of 16 along k:
+ * bscale = E4M3 round-to-nearest-even satfinite of (amax_block / 6) / g;
+ * code = nearest E2M1 of w' / (e4m3(bscale) * g), ties to the even code,
+ * saturating at 6, sign bit = sign of the quotient; all-zero codes when the
+ * block scale is 0.  Bit-for-bit deterministic. */
+int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scale_s,
+                      uint8_t* codes, uint8_t* bscale, float* global_scale, void* stream);
+
+/* awq_search_scale -- AWQ grid search of the per-input-channel scale
+ * ("Lance-Quant" section "量化应用": grid-search AWQ scale equalization;
+ * "quantization primer" section 7: scale salient channels by activation
+ * magnitude).  For each alpha_i:
+ *   a_k = max(mean_t |X[t,k]|, 1e-4)   (or max(act_mean[k], 1e-4) if X == NULL)
+ *   s_k = fp32(a_k ^ alpha_i)
+ *   Delta = W - dequant(Q_int4(W s)) / s     (asymmetric INT4, group_size)
+ *   loss_i = || X Delta^T ||_F^2            (X given, T tokens)
+ *   loss_i = sum_{n,k} (a_k Delta[n,k])^2    (X == NULL: diagonal proxy from
+ *                                             mean |activation| only)
+ *   best = first index of the minimum loss; s_out = s of best.
+ *   W bf16 [N, K]; X bf16 [T, K] or NULL (T > 0 required when X given: an
+ *   empty calibration set is an error); act_mean fp32 [K] used iff X == NULL;
+ *   alphas fp32 [n_alpha] device array; s_out fp32 [K]; loss_out fp32
+ *   [n_alpha]; best_idx int32 [1]; ws/ws_bytes from awq_search_workspace_size.
+ * The chosen s then goes to wq_quantize_int4 / wq_quantize_nvfp4 and its
+ * reciprocal to the linear entry points as act_inv_s. */
+int awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t T,
+                     const float* act_mean, const float* alphas, int n_alpha, int group_size,
+                     float* s_out, float* loss_out, int* best_idx, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* ---------------------------------------------------------------- stage 2: quantized Linear
+ * wq_linear_int4 -- Y = (X * act_inv_s) * dequant(Wq)^T, bf16 in, fp32
+ * accumulate, bf16 out ("quantization primer" sections 4 and 13).
+ *   X        bf16 [M, K]
+ *   qweight/scales/zeros/group_size/zero_point: an INT4 pack from
+ *            wq_quantize_int4 (zeros NULL for symmetric packs)
+ *   act_inv_s fp32 [K] or NULL: multiplies column k of X (the 1/s of an AWQ
+ *            scale that could not be folded into a preceding norm)
+ *   Y        bf16 [M, N]
+ *   ws, ws_bytes: scratch of at least wq_linear_workspace_size bytes (may be
+ *            NULL when that size is 0)
+ * M <= 16 runs the split-K decode GEMV; larger M runs the tensor-core GEMM. */
+int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* qweight,
+                   const uint16_t* scales, const uint32_t* zeros, int group_size, int zero_point,
+                   const float* act_inv_s, uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* wq_linear_nvfp4 -- Y = (X * act_inv_s) * dequant(Wq)^T for an NVFP4 pack.
+ *   act_fp4 = 0: W4A16, activations stay bf16.
+ *   act_fp4 = 1: W4A4 ("OmniQuant" section 4.2): X is first quantized to
+ *            NVFP4 along K with its own per-tensor scale (the
+ *            wq_quantize_nvfp4 rule applied to X), and the product runs on
+ *            the block-scaled FP4 tensor cores; needs workspace.
+ *   other arguments as for wq_linear_int4. */
+int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
+                    const uint8_t* bscale, const float* global_scale, int act_fp4,
+                    const float* act_inv_s, uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronizes `stream`, then reads and clears the device error word of the
+ * current GPU.  WQ_OK if no kernel reported a problem since the last call,
+ * WQ_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the kernel then
+ * exited early and its outputs are undefined), WQ_ERR_CUDA if the stream
+ * itself failed. */
+int wq_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WQ_H_ */

@@ -1,0 +1,81 @@
+"""The C-ABI library: builds for sm_100a, loads, exports every declared symbol,
+and validates arguments on the host (no GPU needed for any of this)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a16_gemm_wq_b200 as wq
+from w4a16_gemm_wq_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "wq.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return wq.load()
+
+
+def test_header_declares_the_five_entry_points():
+    names = declared_functions()
+    for n in ("wq_quantize_int4", "wq_quantize_nvfp4", "awq_search_scale", "wq_linear_int4", "wq_linear_nvfp4"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(wq.SIGNATURES), "binding signatures out of sync with include/wq.h"
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_size_queries(lib):
+    assert wq.int4_sizes(2048, 11008, 128) == (2048 * 11008 // 2, 2048 * 86 * 2, 2048 * 11 * 4)
+    assert wq.int4_sizes(512, 512, 64) == (512 * 256, 512 * 8 * 2, 512 * 1 * 4)
+    assert wq.nvfp4_sizes(2048, 2048) == (2048 * 1024, 2048 * 128)
+    with pytest.raises(wq.WQError) as e:
+        wq.int4_sizes(16, 100, 64)  # K not a multiple of 32
+    assert e.value.status == wq.WQ_ERR_ARG
+    with pytest.raises(wq.WQError) as e:
+        wq.int4_sizes(16, 512, 32)
+    assert e.value.status == wq.WQ_ERR_UNSUPPORTED
+
+
+def _st(lib, rc):
+    return rc, lib.wq_last_error().decode()
+
+
+def test_host_validation_rejects_before_any_launch(lib):
+    P = ctypes.c_void_p
+    good = P(1 << 20)  # 16-byte aligned, never dereferenced: validation fails first
+    bad = P((1 << 20) + 8)
+    # bits != 4 -> unsupported
+    assert lib.wq_quantize_int4(good, 16, 64, 8, 64, 1, None, good, good, good, None) == wq.WQ_ERR_UNSUPPORTED
+    # null input, misaligned output, zeros with a symmetric pack
+    assert lib.wq_quantize_int4(None, 16, 64, 4, 64, 1, None, good, good, good, None) == wq.WQ_ERR_ARG
+    assert lib.wq_quantize_int4(good, 16, 64, 4, 64, 1, None, bad, good, good, None) == wq.WQ_ERR_ARG
+    assert lib.wq_quantize_int4(good, 16, 64, 4, 64, 0, None, good, good, good, None) == wq.WQ_ERR_ARG
+    assert "zeros" in lib.wq_last_error().decode()
+    # K % group_size
+    assert lib.wq_quantize_int4(good, 16, 96, 4, 64, 1, None, good, good, good, None) == wq.WQ_ERR_ARG
+    # empty calibration set is an error ("llm-quantize": reject empty calibration)
+    assert lib.awq_search_scale(good, 16, 64, good, 0, None, good, 20, 64, good, good, good, None, 0, None) \
+        in (wq.WQ_ERR_ARG,)
+    # M <= 0, act_fp4 out of range
+    assert lib.wq_linear_int4(good, 0, 16, 64, good, good, good, 64, 1, None, good, None, 0, None) == wq.WQ_ERR_ARG
+    assert lib.wq_linear_nvfp4(good, 1, 16, 64, good, good, good, 2, None, good, None, 0, None) == wq.WQ_ERR_ARG
+    assert lib.wq_status_string(4).decode().startswith("WQ_ERR_TIMEOUT")
+
+
+def test_binding_refuses_requantizing():
+    p = wq.PackedInt4(None, None, None, 1, 32, 64, 1)
+    with pytest.raises(ValueError):
+        wq.wq_quantize_int4(p)

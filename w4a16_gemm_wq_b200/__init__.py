@@ -1,0 +1,258 @@
+"""B200-native group-wise 4-bit weight-only quantization (INT4 / NVFP4) and the
+quantized Linear Y = X * dequant(Wq)^T.
+
+This module is a thin ctypes binding over ``libwq.so`` (C ABI in
+``include/wq.h``).  It only checks tensor properties and marshals pointers
+and the current CUDA stream; every step of the computation runs in the
+library's CUDA kernels.  There is no CPU fallback: if the library cannot be
+loaded every call raises.
+
+Functions carry the C names:
+    wq_quantize_int4, wq_quantize_nvfp4, awq_search_scale,
+    wq_linear_int4, wq_linear_nvfp4, wq_device_error
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwq.so")
+
+WQ_OK, WQ_ERR_ARG, WQ_ERR_CUDA, WQ_ERR_UNSUPPORTED, WQ_ERR_TIMEOUT = range(5)
+WQ_FMT_INT4, WQ_FMT_NVFP4 = 0, 1
+
+# (name, restype, argtypes) of every symbol declared in include/wq.h
+_P, _I64, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+_PSZ = ctypes.POINTER(ctypes.c_size_t)
+SIGNATURES = {
+    "wq_status_string": (ctypes.c_char_p, [_I]),
+    "wq_last_error": (ctypes.c_char_p, []),
+    "wq_int4_sizes": (_I, [_I64, _I64, _I, _PSZ, _PSZ, _PSZ]),
+    "wq_nvfp4_sizes": (_I, [_I64, _I64, _PSZ, _PSZ]),
+    "wq_linear_workspace_size": (_I, [_I64, _I64, _I64, _I, _I, _PSZ]),
+    "awq_search_workspace_size": (_I, [_I64, _I64, _I64, _I, _I, _PSZ]),
+    "wq_quantize_int4": (_I, [_P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "wq_quantize_nvfp4": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
+    "awq_search_scale": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "wq_linear_int4": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
+    "wq_linear_nvfp4": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]),
+    "wq_device_error": (_I, [_P]),
+}
+
+_lib = None
+
+
+class WQError(RuntimeError):
+    def __init__(self, status: int, where: str, msg: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({msg})")
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load libwq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: build it with `python -m w4a16_gemm_wq_b200.build`")
+    lib = ctypes.CDLL(p)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != WQ_OK:
+        msg = load().wq_last_error().decode(errors="replace")
+        raise WQError(status, where, msg)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _opt_f32(t, name, K):
+    if t is None:
+        return None
+    return _dev(t, name, torch.float32, (K,))
+
+
+# ---------------------------------------------------------------- packed formats
+@dataclasses.dataclass
+class PackedInt4:
+    qweight: torch.Tensor  # int32 view of uint32 [N, K/8]
+    scales: torch.Tensor   # fp16 [N, K/G]
+    zeros: torch.Tensor | None  # int32 view of uint32 [N, ceil(K/G/8)]
+    N: int
+    K: int
+    group_size: int
+    zero_point: int
+
+    def nbytes(self) -> int:
+        z = 0 if self.zeros is None else self.zeros.numel() * 4
+        return self.qweight.numel() * 4 + self.scales.numel() * 2 + z
+
+
+@dataclasses.dataclass
+class PackedNVFP4:
+    codes: torch.Tensor        # uint8 [N, K/2]
+    bscale: torch.Tensor       # uint8 [N, K/16] (E4M3 bits)
+    global_scale: torch.Tensor  # fp32 [1]
+    N: int
+    K: int
+
+    def nbytes(self) -> int:
+        return self.codes.numel() + self.bscale.numel() + 4
+
+
+def int4_sizes(N: int, K: int, group_size: int):
+    q, s, z = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().wq_int4_sizes(N, K, group_size, ctypes.byref(q), ctypes.byref(s), ctypes.byref(z)), "wq_int4_sizes")
+    return q.value, s.value, z.value
+
+
+def nvfp4_sizes(N: int, K: int):
+    c, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().wq_nvfp4_sizes(N, K, ctypes.byref(c), ctypes.byref(b)), "wq_nvfp4_sizes")
+    return c.value, b.value
+
+
+def linear_workspace_size(M: int, N: int, K: int, fmt: int, act_fp4: int = 0) -> int:
+    b = ctypes.c_size_t()
+    _check(load().wq_linear_workspace_size(M, N, K, fmt, act_fp4, ctypes.byref(b)), "wq_linear_workspace_size")
+    return b.value
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------- stage 1
+def wq_quantize_int4(W: torch.Tensor, group_size: int = 64, zero_point: int = 1, scale_s=None,
+                     bits: int = 4) -> PackedInt4:
+    if isinstance(W, (PackedInt4, PackedNVFP4)):
+        raise ValueError("the layer is already quantized")  # "llm-quantize": refuse re-quantizing
+    _dev(W, "W", torch.bfloat16)
+    N, K = W.shape
+    lib = load()
+    ng = K // group_size if group_size and K % group_size == 0 else 1
+    qweight = torch.empty((N, max(K // 8, 1)), dtype=torch.int32, device=W.device)
+    scales = torch.empty((N, ng), dtype=torch.float16, device=W.device)
+    zeros = torch.empty((N, (ng + 7) // 8), dtype=torch.int32, device=W.device) if zero_point else None
+    s = _opt_f32(scale_s, "scale_s", K)
+    _check(lib.wq_quantize_int4(_ptr(W), N, K, bits, group_size, zero_point, _ptr(s), _ptr(qweight),
+                                _ptr(scales), _ptr(zeros), _stream()), "wq_quantize_int4")
+    return PackedInt4(qweight, scales, zeros, N, K, group_size, zero_point)
+
+
+def wq_quantize_nvfp4(W: torch.Tensor, scale_s=None) -> PackedNVFP4:
+    if isinstance(W, (PackedInt4, PackedNVFP4)):
+        raise ValueError("the layer is already quantized")
+    _dev(W, "W", torch.bfloat16)
+    N, K = W.shape
+    lib = load()
+    codes = torch.empty((N, max(K // 2, 1)), dtype=torch.uint8, device=W.device)
+    bscale = torch.empty((N, max(K // 16, 1)), dtype=torch.uint8, device=W.device)
+    g = torch.empty((1,), dtype=torch.float32, device=W.device)
+    s = _opt_f32(scale_s, "scale_s", K)
+    _check(lib.wq_quantize_nvfp4(_ptr(W), N, K, _ptr(s), _ptr(codes), _ptr(bscale), _ptr(g), _stream()),
+           "wq_quantize_nvfp4")
+    return PackedNVFP4(codes, bscale, g, N, K)
+
+
+def awq_search_scale(W: torch.Tensor, alphas: torch.Tensor, group_size: int = 64, X: torch.Tensor | None = None,
+                     act_mean: torch.Tensor | None = None):
+    """Returns (s fp32 [K], losses fp32 [n_alpha], best int32 [1]) as device tensors."""
+    _dev(W, "W", torch.bfloat16)
+    N, K = W.shape
+    T = 0
+    if X is not None:
+        _dev(X, "X", torch.bfloat16)
+        if X.dim() != 2 or X.shape[1] != K:
+            raise ValueError("X must be [T, K]")
+        T = X.shape[0]
+    am = _opt_f32(act_mean, "act_mean", K)
+    _dev(alphas, "alphas", torch.float32)
+    lib = load()
+    n_alpha = alphas.numel()
+    b = ctypes.c_size_t()
+    _check(lib.awq_search_workspace_size(N, K, T, n_alpha, group_size, ctypes.byref(b)), "awq_search_workspace_size")
+    ws = _workspace(b.value, W.device)
+    s = torch.empty(K, dtype=torch.float32, device=W.device)
+    losses = torch.empty(n_alpha, dtype=torch.float32, device=W.device)
+    best = torch.empty(1, dtype=torch.int32, device=W.device)
+    _check(lib.awq_search_scale(_ptr(W), N, K, _ptr(X), T, _ptr(am), _ptr(alphas), n_alpha, group_size, _ptr(s),
+                                _ptr(losses), _ptr(best), _ptr(ws), b.value, _stream()), "awq_search_scale")
+    return s, losses, best
+
+
+# ---------------------------------------------------------------- stage 2
+def wq_linear_int4(X: torch.Tensor, p: PackedInt4, act_inv_s=None, out: torch.Tensor | None = None,
+                   ws: torch.Tensor | None = None) -> torch.Tensor:
+    _dev(X, "X", torch.bfloat16)
+    M, K = X.shape
+    if K != p.K:
+        raise ValueError(f"X has K={K}, the pack K={p.K}")
+    Y = out if out is not None else torch.empty((M, p.N), dtype=torch.bfloat16, device=X.device)
+    _dev(Y, "out", torch.bfloat16, (M, p.N))
+    lib = load()
+    need = linear_workspace_size(M, p.N, K, WQ_FMT_INT4)
+    if ws is None:
+        ws = _workspace(need, X.device)
+    s = _opt_f32(act_inv_s, "act_inv_s", K)
+    _check(lib.wq_linear_int4(_ptr(X), M, p.N, K, _ptr(p.qweight), _ptr(p.scales), _ptr(p.zeros), p.group_size,
+                              p.zero_point, _ptr(s), _ptr(Y), _ptr(ws), 0 if ws is None else ws.numel(), _stream()),
+           "wq_linear_int4")
+    return Y
+
+
+def wq_linear_nvfp4(X: torch.Tensor, p: PackedNVFP4, act_fp4: int = 0, act_inv_s=None,
+                    out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    _dev(X, "X", torch.bfloat16)
+    M, K = X.shape
+    if K != p.K:
+        raise ValueError(f"X has K={K}, the pack K={p.K}")
+    Y = out if out is not None else torch.empty((M, p.N), dtype=torch.bfloat16, device=X.device)
+    _dev(Y, "out", torch.bfloat16, (M, p.N))
+    lib = load()
+    need = linear_workspace_size(M, p.N, K, WQ_FMT_NVFP4, act_fp4)
+    if ws is None:
+        ws = _workspace(need, X.device)
+    s = _opt_f32(act_inv_s, "act_inv_s", K)
+    _check(lib.wq_linear_nvfp4(_ptr(X), M, p.N, K, _ptr(p.codes), _ptr(p.bscale), _ptr(p.global_scale), act_fp4,
+                               _ptr(s), _ptr(Y), _ptr(ws), 0 if ws is None else ws.numel(), _stream()),
+           "wq_linear_nvfp4")
+    return Y
+
+
+def wq_device_error() -> int:
+    """Synchronize the current stream and read/clear the device error word (raises on error)."""
+    st = load().wq_device_error(_stream())
+    _check(st, "wq_device_error")
+    return st

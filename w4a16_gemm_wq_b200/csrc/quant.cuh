@@ -1,0 +1,231 @@
+// quant.cuh -- stage 1 kernels: group-wise INT4 quantize+pack and NVFP4 pack.
+//
+// INT4 rule ("quantization primer", sections 2-3; "OmniQuant" section 2.1):
+// q = clamp(round(w'/scale) + z, 0, 15) per group of G consecutive k with a
+// min-max scale and zero point.  NVFP4 ("Lance-Quant", section "量化应用";
+// "quantization primer", section 12): E2M1 codes, one E4M3 scale per 16 k,
+// one fp32 scale per tensor.  Every decision is taken in fp32 with IEEE
+// round-to-nearest-even arithmetic (__fdiv_rn / __fmul_rn, never fused) so
+// the packed bytes are bit-exact and reproducible.
+//
+// Both kernels are HBM-bound streaming passes: each thread reads 16 bytes
+// (8 bf16) with one 128-bit load and writes one 32-bit word of codes.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "wq_common.cuh"
+
+namespace wq {
+
+// ------------------------------------------------------------------ INT4
+constexpr int kQuantThreads = 256;  // one row chunk of 256 * 8 = 2048 k per CTA
+
+// Loads 8 consecutive bf16 weights of row n starting at k (k % 8 == 0) and
+// applies the optional per-channel AWQ scale (one fp32 multiply each).
+__device__ __forceinline__ void load_wprime8(const uint16_t* __restrict__ W, const float* __restrict__ s,
+                                             int64_t K, int64_t n, int64_t k, float w[8]) {
+  const uint4 v = ldg_stream_v4(W + n * K + k);
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    w[2 * j] = __uint_as_float(u[j] << 16);
+    w[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
+  }
+  if (s) {
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + k));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + k + 4));
+    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = __fmul_rn(w[j], sv[j]);
+  }
+}
+
+// fp16 scale of a group from its fp32 range: clamp(r / levels, 1e-5, 65504),
+// rounded to nearest even.  Returns the fp16 bits; *sc is its value.
+__device__ __forceinline__ uint16_t group_scale_f16(float r, float levels, float* sc) {
+  float sc32 = __fdiv_rn(r, levels);
+  if (!(sc32 >= 1e-5f)) sc32 = 1e-5f;
+  if (sc32 > 65504.0f) sc32 = 65504.0f;
+  const __half h = __float2half_rn(sc32);
+  *sc = __half2float(h);
+  return __half_as_ushort(h);
+}
+
+// grid = (ceil(K/2048), N); thread t of CTA (c, n) owns word u = c*256 + t of
+// row n, i.e. k in [8u, 8u+8).  A group is G/8 consecutive lanes of one warp.
+template <int G, bool ASYM>
+__global__ void __launch_bounds__(kQuantThreads) quantize_int4_kernel(
+    const uint16_t* __restrict__ W, const float* __restrict__ s, int64_t N, int64_t K,
+    uint32_t* __restrict__ qweight, uint16_t* __restrict__ scales, uint32_t* __restrict__ zeros) {
+  constexpr int LPG = G / 8;  // lanes per group
+  __shared__ uint8_t zsh[kQuantThreads / LPG];
+  const int64_t n = blockIdx.y;
+  const int64_t words = K / 8;
+  const int64_t u = int64_t(blockIdx.x) * kQuantThreads + threadIdx.x;
+  const bool active = u < words;
+  const int64_t k = u * 8;
+
+  float w[8];
+  float mn = INFINITY, mx = -INFINITY, amax = 0.f;
+  if (active) {
+    load_wprime8(W, s, K, n, k, w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      mn = fminf(mn, w[j]);
+      mx = fmaxf(mx, w[j]);
+      amax = fmaxf(amax, fabsf(w[j]));
+    }
+  }
+  // groups never straddle a warp (LPG divides 32, rows hold whole groups)
+#pragma unroll
+  for (int off = 1; off < LPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  }
+  const int64_t ng = K / G;
+  const int64_t g = k / G;
+  float sc, z = 0.f;
+  uint16_t hbits;
+  if (ASYM) {
+    hbits = group_scale_f16(__fsub_rn(mx, mn), 15.0f, &sc);
+    z = fminf(fmaxf(rintf(__fdiv_rn(-mn, sc)), 0.0f), 15.0f);
+  } else {
+    hbits = group_scale_f16(amax, 7.0f, &sc);
+  }
+  if (active) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float r = rintf(__fdiv_rn(w[j], sc));
+      const float q = ASYM ? fminf(fmaxf(__fadd_rn(r, z), 0.0f), 15.0f)
+                           : __fadd_rn(fminf(fmaxf(r, -7.0f), 7.0f), 8.0f);
+      word |= uint32_t(q) << (4 * j);
+    }
+    qweight[n * words + u] = word;
+    if ((threadIdx.x % LPG) == 0) scales[n * ng + g] = hbits;
+  }
+  if (ASYM) {
+    // Pack 8 group zero points per word.  A CTA covers 2048 k of one row,
+    // a whole number of zero words (8*G divides 2048), so no word is shared.
+    if ((threadIdx.x % LPG) == 0) zsh[threadIdx.x / LPG] = active ? uint8_t(z) : uint8_t(0);
+    __syncthreads();
+    constexpr int GROUPS_PER_CTA = kQuantThreads / LPG;
+    const int64_t nzw = (ng + 7) / 8;
+    const int64_t g0 = int64_t(blockIdx.x) * GROUPS_PER_CTA;
+    if (threadIdx.x < GROUPS_PER_CTA / 8) {
+      const int64_t zw = g0 / 8 + threadIdx.x;
+      if (zw < nzw) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int64_t gg = zw * 8 + j;
+          if (gg < ng) word |= uint32_t(zsh[threadIdx.x * 8 + j] & 0xF) << (4 * j);
+        }
+        zeros[n * nzw + zw] = word;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ NVFP4
+// Round-to-nearest-even of a non-negative finite fp32 to E4M3, saturating
+// at 448 (code 0x7E).  Bit-level rounding of the fp32 significand.
+__device__ __forceinline__ uint32_t e4m3_encode_satfinite(float t) {
+  if (!(t < 448.0f)) return 0x7E;          // also catches +inf
+  const uint32_t bits = __float_as_uint(t);
+  const int E = int(bits >> 23) - 127;
+  if (E < -6) {                            // below 2^-6: subnormal grid m * 2^-9
+    const float m = rintf(t * 512.0f);       // exact scaling, RNE
+    return uint32_t(m);                      // m == 8 encodes 2^-6 = code 0x08
+  }
+  uint32_t e = uint32_t(E + 7);
+  const uint32_t man = bits & 0x7FFFFFu;
+  uint32_t keep = man >> 20;
+  const uint32_t rem = man & 0xFFFFFu;
+  if (rem > 0x80000u || (rem == 0x80000u && (keep & 1u))) ++keep;
+  if (keep == 8) { keep = 0; ++e; }
+  if (e > 15 || (e == 15 && keep == 7)) return 0x7E;
+  return (e << 3) | keep;
+}
+
+// Nearest E2M1 code of v (ties to the even code, saturating at 6, sign bit
+// from v).  Magnitudes by code: 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ uint32_t e2m1_encode(float v) {
+  const float a = fabsf(v);
+  uint32_t c;
+  if (a <= 0.25f) c = 0;
+  else if (a < 0.75f) c = 1;
+  else if (a <= 1.25f) c = 2;
+  else if (a < 1.75f) c = 3;
+  else if (a <= 2.5f) c = 4;
+  else if (a < 3.5f) c = 5;
+  else if (a <= 5.0f) c = 6;
+  else c = 7;
+  return c | ((__float_as_uint(v) >> 28) & 8u);
+}
+
+// Pass 1: amax over the tensor, atomically max-ed into *amax_out (which the
+// host zeroed).  Non-negative floats order like their bit patterns.
+__global__ void __launch_bounds__(256) nvfp4_amax_kernel(const uint16_t* __restrict__ A, const float* __restrict__ s,
+                                                         int64_t R, int64_t C, float* amax_out) {
+  const int64_t words = R * C / 8;
+  float m = 0.f;
+  for (int64_t u = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u < words; u += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = (u * 8) / C, c = (u * 8) % C;
+    float w[8];
+    load_wprime8(A, s, C, r, c, w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(w[j]));
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < int(blockDim.x >> 5); ++i) m = fmaxf(m, red[i]);
+    atomicMax(reinterpret_cast<unsigned int*>(amax_out), __float_as_uint(m));
+  }
+}
+
+__device__ __forceinline__ float nvfp4_global_from_amax(float amax) {
+  return amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f;  // 6 * 448
+}
+
+// Pass 2: one thread per block of 16 consecutive elements (flat order), so
+// block-scale bytes and 8-byte code groups are written coalesced.
+__global__ void __launch_bounds__(256) nvfp4_pack_kernel(const uint16_t* __restrict__ A, const float* __restrict__ s,
+                                                         int64_t R, int64_t C, const float* __restrict__ amax_in,
+                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ bscale) {
+  const int64_t nblk = R * C / 16;
+  const float g = nvfp4_global_from_amax(*amax_in);
+  for (int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; b < nblk; b += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = (b * 16) / C, c = (b * 16) % C;
+    float w[16];
+    load_wprime8(A, s, C, r, c, w);
+    load_wprime8(A, s, C, r, c + 8, w + 8);
+    float ab = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) ab = fmaxf(ab, fabsf(w[j]));
+    const float t = __fdiv_rn(__fdiv_rn(ab, 6.0f), g);
+    const uint32_t sb = e4m3_encode_satfinite(t);
+    const float d = e4m3_decode_pos(sb);
+    uint32_t lo = 0, hi = 0;
+    if (d != 0.0f) {
+      const float denom = __fmul_rn(d, g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) lo |= e2m1_encode(__fdiv_rn(w[j], denom)) << (4 * j);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) hi |= e2m1_encode(__fdiv_rn(w[8 + j], denom)) << (4 * j);
+    }
+    reinterpret_cast<uint2*>(codes)[b] = make_uint2(lo, hi);
+    bscale[b] = uint8_t(sb);
+  }
+}
+
+// Pass 3: replace the amax in *gs by the per-tensor scale g.
+__global__ void nvfp4_finalize_kernel(float* gs) { *gs = nvfp4_global_from_amax(*gs); }
+
+}  // namespace wq

@@ -1,0 +1,300 @@
+// wq_api.cu -- host side of libwq: argument validation, launch configuration
+// and the extern "C" entry points declared in include/wq.h.  All kernels are
+// compiled into this one translation unit for sm_100a.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "../../include/wq.h"
+#include "gemv.cuh"
+#include "quant.cuh"
+#include "wq_common.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int status, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return status;
+}
+
+int cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return WQ_OK;
+  return fail(WQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE(cond, ...)                         \
+  do {                                             \
+    if (!(cond)) return fail(WQ_ERR_ARG, __VA_ARGS__); \
+  } while (0)
+
+#define REQUIRE_PTR(p)                                                        \
+  do {                                                                        \
+    if (!(p)) return fail(WQ_ERR_ARG, "%s must not be NULL", #p);             \
+    if (!aligned16(p)) return fail(WQ_ERR_ARG, "%s must be 16-byte aligned", #p); \
+  } while (0)
+
+#define REQUIRE_OPT_PTR(p)                                                    \
+  do {                                                                        \
+    if ((p) && !aligned16(p)) return fail(WQ_ERR_ARG, "%s must be 16-byte aligned", #p); \
+  } while (0)
+
+int check_shape(int64_t N, int64_t K) {
+  REQUIRE(N > 0 && K > 0, "N and K must be positive (got N=%lld K=%lld)", (long long)N, (long long)K);
+  REQUIRE(K % 32 == 0, "K must be a multiple of 32 (got %lld)", (long long)K);
+  REQUIRE(N <= (int64_t(1) << 30) && K <= (int64_t(1) << 30), "N and K must be below 2^30");
+  return WQ_OK;
+}
+
+int check_group(int group_size, int64_t K) {
+  if (group_size != 64 && group_size != 128)
+    return fail(WQ_ERR_UNSUPPORTED, "group_size must be 64 or 128 (got %d)", group_size);
+  REQUIRE(K % group_size == 0, "K (%lld) must be a multiple of group_size (%d)", (long long)K, group_size);
+  return WQ_OK;
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int launched(const char* what) { return cuda_check(cudaGetLastError(), what); }
+
+// ---------------------------------------------------------------- GEMV launch
+template <int FMT, int MT>
+int launch_gemv_mt(const wq::GemvArgs& a0, cudaStream_t st) {
+  wq::GemvArgs a = a0;
+  const int rows_per_cta = wq::kGemvWarps * wq::kGemvRows;
+  const int gx = (a.N + rows_per_cta - 1) / rows_per_cta;
+  const int gz = (a.M + MT - 1) / MT;
+  const int iters = (a.K + wq::kGemvKPerIter - 1) / wq::kGemvKPerIter;
+  int splits = (2 * 148 + gx * gz - 1) / (gx * gz);
+  splits = std::max(1, std::min({splits, wq::kGemvMaxSplits, iters}));
+  a.iters_per_split = (iters + splits - 1) / splits;
+  splits = (iters + a.iters_per_split - 1) / a.iters_per_split;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(gx, splits, gz);
+  cfg.blockDim = dim3(wq::kGemvWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = splits;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = splits > 1 ? 1 : 0;
+  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemv_kernel<FMT, MT>, a), "gemv launch");
+}
+
+template <int FMT>
+int launch_gemv(const wq::GemvArgs& a, cudaStream_t st) {
+  if (a.M == 1) return launch_gemv_mt<FMT, 1>(a, st);
+  if (a.M == 2) return launch_gemv_mt<FMT, 2>(a, st);
+  return launch_gemv_mt<FMT, 4>(a, st);
+}
+
+int log2i(int v) {
+  int r = 0;
+  while ((1 << r) < v) ++r;
+  return r;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* wq_status_string(int status) {
+  switch (status) {
+    case WQ_OK: return "WQ_OK";
+    case WQ_ERR_ARG: return "WQ_ERR_ARG (invalid argument)";
+    case WQ_ERR_CUDA: return "WQ_ERR_CUDA (CUDA runtime failure)";
+    case WQ_ERR_UNSUPPORTED: return "WQ_ERR_UNSUPPORTED (unsupported parameters)";
+    case WQ_ERR_TIMEOUT: return "WQ_ERR_TIMEOUT (device-side wait gave up)";
+    default: return "unknown wq status";
+  }
+}
+
+const char* wq_last_error(void) { return g_last_error; }
+
+int wq_int4_sizes(int64_t N, int64_t K, int group_size, size_t* qweight_bytes, size_t* scales_bytes,
+                  size_t* zeros_bytes) {
+  if (int e = check_shape(N, K)) return e;
+  if (int e = check_group(group_size, K)) return e;
+  const int64_t ng = K / group_size;
+  if (qweight_bytes) *qweight_bytes = size_t(N) * size_t(K / 8) * 4;
+  if (scales_bytes) *scales_bytes = size_t(N) * size_t(ng) * 2;
+  if (zeros_bytes) *zeros_bytes = size_t(N) * size_t((ng + 7) / 8) * 4;
+  return WQ_OK;
+}
+
+int wq_nvfp4_sizes(int64_t N, int64_t K, size_t* codes_bytes, size_t* bscale_bytes) {
+  if (int e = check_shape(N, K)) return e;
+  if (codes_bytes) *codes_bytes = size_t(N) * size_t(K / 2);
+  if (bscale_bytes) *bscale_bytes = size_t(N) * size_t(K / 16);
+  return WQ_OK;
+}
+
+int wq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int format, int act_fp4, size_t* bytes) {
+  REQUIRE(bytes, "bytes must not be NULL");
+  REQUIRE(M > 0, "M must be positive");
+  if (int e = check_shape(N, K)) return e;
+  REQUIRE(format == WQ_FMT_INT4 || format == WQ_FMT_NVFP4, "unknown format %d", format);
+  *bytes = 0;
+  (void)act_fp4;
+  return WQ_OK;
+}
+
+int awq_search_workspace_size(int64_t N, int64_t K, int64_t T, int n_alpha, int group_size, size_t* bytes) {
+  REQUIRE(bytes, "bytes must not be NULL");
+  if (int e = check_shape(N, K)) return e;
+  if (int e = check_group(group_size, K)) return e;
+  (void)T;
+  (void)n_alpha;
+  *bytes = 0;
+  return fail(WQ_ERR_UNSUPPORTED, "awq_search_scale is not available in this build");
+}
+
+int wq_quantize_int4(const uint16_t* W, int64_t N, int64_t K, int bits, int group_size, int zero_point,
+                     const float* scale_s, uint32_t* qweight, uint16_t* scales, uint32_t* zeros, void* stream) {
+  if (bits != 4) return fail(WQ_ERR_UNSUPPORTED, "bits must be 4 (got %d)", bits);
+  if (int e = check_shape(N, K)) return e;
+  if (int e = check_group(group_size, K)) return e;
+  REQUIRE(zero_point == 0 || zero_point == 1, "zero_point must be 0 or 1");
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(qweight);
+  REQUIRE_PTR(scales);
+  REQUIRE_OPT_PTR(scale_s);
+  if (zero_point) {
+    REQUIRE_PTR(zeros);
+  } else {
+    REQUIRE(!zeros, "zeros must be NULL for a symmetric (zero_point=0) pack");
+  }
+  const dim3 grid(unsigned((K / 8 + wq::kQuantThreads - 1) / wq::kQuantThreads), unsigned(N));
+  cudaStream_t st = as_stream(stream);
+  if (group_size == 64) {
+    if (zero_point)
+      wq::quantize_int4_kernel<64, true><<<grid, wq::kQuantThreads, 0, st>>>(W, scale_s, N, K, qweight, scales, zeros);
+    else
+      wq::quantize_int4_kernel<64, false><<<grid, wq::kQuantThreads, 0, st>>>(W, scale_s, N, K, qweight, scales, zeros);
+  } else {
+    if (zero_point)
+      wq::quantize_int4_kernel<128, true><<<grid, wq::kQuantThreads, 0, st>>>(W, scale_s, N, K, qweight, scales, zeros);
+    else
+      wq::quantize_int4_kernel<128, false><<<grid, wq::kQuantThreads, 0, st>>>(W, scale_s, N, K, qweight, scales, zeros);
+  }
+  return launched("quantize_int4 launch");
+}
+
+int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scale_s, uint8_t* codes,
+                      uint8_t* bscale, float* global_scale, void* stream) {
+  if (int e = check_shape(N, K)) return e;
+  REQUIRE_PTR(W);
+  REQUIRE_PTR(codes);
+  REQUIRE_PTR(bscale);
+  REQUIRE_PTR(global_scale);
+  REQUIRE_OPT_PTR(scale_s);
+  cudaStream_t st = as_stream(stream);
+  // global_scale first accumulates amax, then the pack pass reads it, then it
+  // is replaced by g: three stream-ordered steps, no scratch memory.
+  if (int e = cuda_check(cudaMemsetAsync(global_scale, 0, sizeof(float), st), "memset")) return e;
+  const int64_t words = N * K / 8;
+  const int amax_blocks = int(std::min<int64_t>((words + 255) / 256, 148 * 8));
+  wq::nvfp4_amax_kernel<<<amax_blocks, 256, 0, st>>>(W, scale_s, N, K, global_scale);
+  if (int e = launched("nvfp4_amax launch")) return e;
+  const int64_t nblk = N * K / 16;
+  const int pack_blocks = int(std::min<int64_t>((nblk + 255) / 256, 148 * 16));
+  wq::nvfp4_pack_kernel<<<pack_blocks, 256, 0, st>>>(W, scale_s, N, K, global_scale, codes, bscale);
+  if (int e = launched("nvfp4_pack launch")) return e;
+  wq::nvfp4_finalize_kernel<<<1, 1, 0, st>>>(global_scale);
+  return launched("nvfp4_finalize launch");
+}
+
+int awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t T, const float* act_mean,
+                     const float* alphas, int n_alpha, int group_size, float* s_out, float* loss_out, int* best_idx,
+                     void* ws, size_t ws_bytes, void* stream) {
+  if (int e = check_shape(N, K)) return e;
+  if (int e = check_group(group_size, K)) return e;
+  REQUIRE_PTR(W);
+  if (X) {
+    REQUIRE_PTR(X);
+    REQUIRE(T > 0, "empty calibration set: X given with T=%lld tokens", (long long)T);
+  } else {
+    REQUIRE(act_mean, "either X (calibration tokens) or act_mean is required");
+    REQUIRE_PTR(act_mean);
+  }
+  REQUIRE(n_alpha > 0 && n_alpha <= 1024, "n_alpha must be in 1..1024");
+  REQUIRE_PTR(alphas);
+  REQUIRE_PTR(s_out);
+  REQUIRE_PTR(loss_out);
+  REQUIRE_PTR(best_idx);
+  (void)ws; (void)ws_bytes; (void)stream;
+  return fail(WQ_ERR_UNSUPPORTED, "awq_search_scale is not available in this build");
+}
+
+int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* qweight,
+                   const uint16_t* scales, const uint32_t* zeros, int group_size, int zero_point,
+                   const float* act_inv_s, uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  REQUIRE(M > 0 && M <= (int64_t(1) << 30), "M must be positive");
+  if (int e = check_shape(N, K)) return e;
+  if (int e = check_group(group_size, K)) return e;
+  REQUIRE(zero_point == 0 || zero_point == 1, "zero_point must be 0 or 1");
+  REQUIRE_PTR(X);
+  REQUIRE_PTR(qweight);
+  REQUIRE_PTR(scales);
+  REQUIRE_PTR(Y);
+  REQUIRE_OPT_PTR(act_inv_s);
+  if (zero_point) {
+    REQUIRE_PTR(zeros);
+  } else {
+    REQUIRE(!zeros, "zeros must be NULL for a symmetric (zero_point=0) pack");
+  }
+  wq::GemvArgs a = {};
+  a.X = X; a.inv_s = act_inv_s; a.wq = qweight; a.scales = scales; a.zeros = zeros;
+  a.Y = Y; a.M = int(M); a.N = int(N); a.K = int(K); a.log2g = log2i(group_size);
+  return launch_gemv<wq::FMT_INT4>(a, as_stream(stream));
+}
+
+int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
+                    const uint8_t* bscale, const float* global_scale, int act_fp4, const float* act_inv_s,
+                    uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  REQUIRE(M > 0 && M <= (int64_t(1) << 30), "M must be positive");
+  if (int e = check_shape(N, K)) return e;
+  REQUIRE(act_fp4 == 0 || act_fp4 == 1, "act_fp4 must be 0 or 1");
+  if (act_fp4) return fail(WQ_ERR_UNSUPPORTED, "W4A4 (act_fp4=1) is not available in this build");
+  REQUIRE_PTR(X);
+  REQUIRE_PTR(codes);
+  REQUIRE_PTR(bscale);
+  REQUIRE_PTR(global_scale);
+  REQUIRE_PTR(Y);
+  REQUIRE_OPT_PTR(act_inv_s);
+  wq::GemvArgs a = {};
+  a.X = X; a.inv_s = act_inv_s; a.wq = codes; a.bscale = bscale; a.gscale = global_scale;
+  a.Y = Y; a.M = int(M); a.N = int(N); a.K = int(K);
+  return launch_gemv<wq::FMT_NVFP4>(a, as_stream(stream));
+}
+
+int wq_device_error(void* stream) {
+  cudaStream_t st = as_stream(stream);
+  if (int e = cuda_check(cudaStreamSynchronize(st), "stream synchronize")) return e;
+  unsigned word = 0;
+  if (int e = cuda_check(cudaMemcpyFromSymbol(&word, wq::g_error_word, sizeof word), "read error word")) return e;
+  if (!word) return WQ_OK;
+  const unsigned zero = 0;
+  if (int e = cuda_check(cudaMemcpyToSymbol(wq::g_error_word, &zero, sizeof zero), "clear error word")) return e;
+  return fail(WQ_ERR_TIMEOUT, "device error word 0x%x (1=TMA wait, 2=MMA wait, 4=pipeline wait, 8=bounds)", word);
+}
+
+}  // extern "C"
