@@ -1,0 +1,92 @@
+"""Prefill GEMM parity (M > 16, tcgen05 tensor cores): outputs against the
+oracle's fp64 product of the same dequantized weights, on all rows for small
+problems and on sampled rows (every tile row band plus the ragged tail) at
+the full transformer-block shapes."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w4a16_gemm_wq_b200 import synth
+from tests._parity import assert_linear_close
+from tests.test_gpu_gemv import _ref_int4, _ref_nvfp4
+
+pytestmark = pytest.mark.gpu
+
+
+def _deq(p):
+    if hasattr(p, "qweight"):
+        return oracle.dequant_int4(dict(qweight=p.qweight.cpu().numpy().view(np.uint32),
+                                        scales=p.scales.cpu().view(torch.int16).numpy().view(np.uint16),
+                                        zeros=None if p.zeros is None else p.zeros.cpu().numpy().view(np.uint32),
+                                        N=p.N, K=p.K, group_size=p.group_size, zero_point=p.zero_point))
+    return oracle.dequant_nvfp4(dict(codes=p.codes.cpu().numpy(), bscale=p.bscale.cpu().numpy(),
+                                     g=p.global_scale.cpu().numpy()[0], N=p.N, K=p.K))
+
+
+@pytest.mark.parametrize("M", [17, 64, 128, 129, 200, 512])
+@pytest.mark.parametrize("fmt", ["int4_g64", "int4_g128", "int4_sym", "nvfp4"])
+def test_small_gemm_all_rows(lib, M, fmt):
+    K, N = 512, 384  # 3 N-tiles of 128, ragged M tiles
+    W = synth.weight(N, K, seed=M)
+    X = synth.activations(M, K, seed=M + 1)
+    if fmt == "nvfp4":
+        p = lib.wq_quantize_nvfp4(W.cuda())
+        Y = lib.wq_linear_nvfp4(X.cuda(), p)
+        ref = _ref_nvfp4(p, X)
+    else:
+        G = 128 if fmt == "int4_g128" else 64
+        p = lib.wq_quantize_int4(W.cuda(), G, 0 if fmt == "int4_sym" else 1)
+        Y = lib.wq_linear_int4(X.cuda(), p)
+        ref = _ref_int4(p, X)
+    assert_linear_close(Y, ref, what=f"{fmt} M={M}")
+
+
+@pytest.mark.parametrize("K,N", [(96, 40), (1056, 200), (2048, 520)])
+def test_ragged_k_and_n(lib, K, N):
+    M = 160
+    W = synth.weight(N, K, seed=K)
+    X = synth.activations(M, K, seed=N)
+    inv_s = synth.act_mean_lognormal(K, seed=K).numpy().astype(np.float32)
+    p = lib.wq_quantize_nvfp4(W.cuda())
+    Y = lib.wq_linear_nvfp4(X.cuda(), p, act_inv_s=torch.tensor(inv_s).cuda())
+    assert_linear_close(Y, _ref_nvfp4(p, X, inv_s), what=f"nvfp4 {K}x{N}")
+    if K % 64 == 0:
+        p = lib.wq_quantize_int4(W.cuda(), 64, 1)
+        Y = lib.wq_linear_int4(X.cuda(), p, act_inv_s=torch.tensor(inv_s).cuda())
+        assert_linear_close(Y, _ref_int4(p, X, inv_s), what=f"int4 {K}x{N}")
+
+
+def _sampled_rows(M, n=24):
+    rows = set(range(0, M, max(1, M // n)))
+    rows.update({0, 127, 128, M - 1})
+    return np.array(sorted(r for r in rows if r < M))
+
+
+@pytest.mark.parametrize("name,K,N", [p for p in synth.PROJECTIONS if p[0] in ("q_proj", "k_proj", "gate_proj", "down_proj")])
+@pytest.mark.parametrize("M", [512, 2048])
+@pytest.mark.parametrize("fmt", ["int4_g64", "nvfp4"])
+def test_config4_block_projection_sampled(lib, name, K, N, M, fmt):
+    W = synth.weight(N, K, seed=synth.layer_seed(4, K + N), device="cuda")
+    X = synth.activations(M, K, seed=synth.layer_seed(4, M), device="cuda")
+    if fmt == "nvfp4":
+        p = lib.wq_quantize_nvfp4(W)
+        Y = lib.wq_linear_nvfp4(X, p)
+    else:
+        p = lib.wq_quantize_int4(W, 64, 1)
+        Y = lib.wq_linear_int4(X, p)
+    rows = _sampled_rows(M)
+    ref = oracle.linear(X[rows].cpu(), _deq(p))
+    assert_linear_close(Y[rows], ref, what=f"{fmt} {name} M={M}")
+
+
+def test_m8192_gate_sampled(lib):
+    K, N, M = 2048, 11008, 8192
+    W = synth.weight(N, K, seed=99, device="cuda")
+    X = synth.activations(M, K, seed=98, device="cuda")
+    p = lib.wq_quantize_int4(W, 64, 1)
+    Y = lib.wq_linear_int4(X, p)
+    rows = _sampled_rows(M, 16)
+    ref = oracle.linear(X[rows].cpu(), _deq(p))
+    assert_linear_close(Y[rows], ref, what="int4 gate M=8192")
+    assert lib.wq_device_error() == 0

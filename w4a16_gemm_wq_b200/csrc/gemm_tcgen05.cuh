@@ -1,0 +1,383 @@
+// gemm_tcgen05.cuh -- prefill GEMM for the quantized Linear at large M on the
+// 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// Y[M, N] = (X * act_inv_s)[M, K] * dequant(Wq)[N, K]^T, bf16 x bf16 -> fp32
+// accumulate in tensor memory -> bf16.  This is the fused alternative the
+// pages call for ("quantization primer" section 13: read compressed weights,
+// dequantize inside the kernel, multiply; "Lance-Quant" section "当前局限":
+// a pure dequant-then-matmul module is ~10% slower than bf16).
+//
+// One CTA computes one BM x BN output tile (BM = 128 rows of X, BN = 128 or
+// 256 rows of W) with warp-specialized roles and an mbarrier pipeline of
+// STAGES k-blocks (BK = 64):
+//   warp 0      TMA producer: X tile [BM x 64] bf16 (128-byte swizzle) and
+//               the packed weight tile [BN x 32 bytes] into stage s;
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//               (M=128, N=BN, K=16, four per k-block), tcgen05.commit frees
+//               the stage and finally signals the epilogue;
+//   warps 4..   BN dequantizer threads, one weight row each: unpack 64
+//               codes of the stage to bf16 (INT4: (q - z) * scale; NVFP4:
+//               e2m1 * e4m3 block scale, the fp32 tensor scale is applied in
+//               the epilogue) and store them in the canonical K-major
+//               128-byte-swizzled layout the MMA reads; then, after the last
+//               k-block, the same warps drain the accumulator with
+//               tcgen05.ld and write bf16 rows of Y.
+// Every wait is bounded (2 s): a stuck pipeline sets the device error word
+// and the CTA leaves after releasing its tensor memory.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "wq_common.cuh"
+
+namespace wq {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 64;
+
+template <int BN>
+struct GemmShape {
+  static constexpr int STAGES = (BN == 256) ? 3 : 4;
+  static constexpr int A_BYTES = kGemmBM * kGemmBK * 2;  // 16 KB, bf16 X tile
+  static constexpr int B_BYTES = BN * kGemmBK * 2;       // dequantized W tile
+  static constexpr int P_BYTES = BN * kGemmBK / 2;       // packed 4-bit W tile
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
+  static constexpr int DEQ_THREADS = BN;
+  static constexpr int THREADS = 128 + DEQ_THREADS;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+};
+
+struct GemmArgs {
+  CUtensorMap tmA;          // X bf16 [M, K]: dims {K, M}, box {64, 128}, 128B swizzle
+  CUtensorMap tmP;          // packed codes u8 [N, K/2]: dims {K/2, N}, box {32, BN}
+  const uint16_t* scales;   // INT4 fp16 [N, K/G]
+  const uint32_t* zeros;    // INT4 [N, ceil(K/G/8)] or null (symmetric, z = 8)
+  const uint8_t* bscale;    // NVFP4 e4m3 [N, K/16]
+  const float* gscale;      // NVFP4 fp32 [1]
+  const float* inv_s;       // fp32 [K] or null
+  uint16_t* Y;              // bf16 [M, N]
+  int M, N, K;
+  int log2g;
+};
+
+// ------------------------------------------------------------------ tcgen05 helpers
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulator.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on `bar` once every previously issued tcgen05.mma of this thread completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile in the canonical
+// 128-byte-swizzle layout: 8-row x 128-byte atoms, atoms 1024 B apart.
+__device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFFu);  // start address
+  d |= uint64_t(1) << 16;                 // leading byte offset (unused by swizzled K-major)
+  d |= uint64_t(1024 >> 4) << 32;         // stride byte offset: next 8-row atom
+  d |= uint64_t(1) << 46;                 // descriptor version of sm_100
+  d |= uint64_t(2) << 61;                 // 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// 32 lanes x 32 columns of fp32 from tensor memory (this warp's lane quarter).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hmul2(*reinterpret_cast<__nv_bfloat162*>(&a), *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t prmt_b32(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ uint32_t lop3_andor(uint32_t a, uint32_t mask, uint32_t bits) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(mask), "r"(bits));
+  return d;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// Byte offset of 16-byte chunk `c` (k = 8c..8c+7) of row `r` in a K-major
+// 128B-swizzled tile (rows of 128 bytes, 8-row atoms of 1024 bytes).
+__device__ __forceinline__ uint32_t sw128_offset(int r, int c) {
+  return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// INT4: one packed word (codes of k = 8j..8j+7) -> 8 bf16 (q - z) * scale,
+// natural k order, as 4 bf16x2 words.
+__device__ __forceinline__ uint4 dequant_word_int4(uint32_t w, uint32_t zoff2, uint32_t sc2) {
+  // {128 + q_i, 128 + q_{i+4}} for i = 0..3 (bf16 exponent-bias trick), exact
+  uint32_t p0 = lop3_andor(w, 0x000F000Fu, 0x43004300u);
+  uint32_t p1 = lop3_andor(w >> 4, 0x000F000Fu, 0x43004300u);
+  uint32_t p2 = lop3_andor(w >> 8, 0x000F000Fu, 0x43004300u);
+  uint32_t p3 = lop3_andor(w >> 12, 0x000F000Fu, 0x43004300u);
+  // (128 + q) - (128 + z) = q - z exactly, then * scale (one bf16 rounding)
+  p0 = bf16x2_mul(bf16x2_sub(p0, zoff2), sc2);
+  p1 = bf16x2_mul(bf16x2_sub(p1, zoff2), sc2);
+  p2 = bf16x2_mul(bf16x2_sub(p2, zoff2), sc2);
+  p3 = bf16x2_mul(bf16x2_sub(p3, zoff2), sc2);
+  // p_i = {w_i, w_{i+4}} -> natural pairs {w0,w1} {w2,w3} {w4,w5} {w6,w7}
+  return make_uint4(prmt_b32(p0, p1, 0x5410), prmt_b32(p2, p3, 0x5410), prmt_b32(p0, p1, 0x7632),
+                    prmt_b32(p2, p3, 0x7632));
+}
+
+// NVFP4: one packed word (codes of k = 8j..8j+7, low nibble = even k) -> 8 bf16
+// e2m1 * sb (exact in bf16), natural order.
+__device__ __forceinline__ uint32_t e2m1x2_to_bf16x2_scaled(uint32_t byte, float sb) {
+  uint32_t h;
+  asm("{ .reg .b8 q; cvt.u8.u32 q, %1; cvt.rn.f16x2.e2m1x2 %0, q; }" : "=r"(h) : "r"(byte));
+  const __half2 hh = *reinterpret_cast<const __half2*>(&h);
+  const float2 f = __half22float2(hh);
+  return pack_bf16x2(f.x * sb, f.y * sb);
+}
+__device__ __forceinline__ uint4 dequant_word_nvfp4(uint32_t w, float sb) {
+  return make_uint4(e2m1x2_to_bf16x2_scaled(w & 0xFF, sb), e2m1x2_to_bf16x2_scaled((w >> 8) & 0xFF, sb),
+                    e2m1x2_to_bf16x2_scaled((w >> 16) & 0xFF, sb), e2m1x2_to_bf16x2_scaled(w >> 24, sb));
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+template <int FMT, int BN>
+__global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel(const __grid_constant__ GemmArgs a) {
+  using S = GemmShape<BN>;
+  constexpr int STAGES = S::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled operand tiles
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  const uint32_t sbase = smem_u32(smem);
+  // stage s: A at s*STAGE, B after A, P after B
+  auto a_addr = [&](int s) { return sbase + uint32_t(s * S::STAGE_BYTES); };
+  auto b_addr = [&](int s) { return sbase + uint32_t(s * S::STAGE_BYTES + S::A_BYTES); };
+  auto p_ptr = [&](int s) { return smem + s * S::STAGE_BYTES + S::A_BYTES + S::B_BYTES; };
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+  uint64_t* full = bars;                 // TMA landed (A + packed W)
+  uint64_t* bready = bars + STAGES;      // dequantized W written
+  uint64_t* empty = bars + 2 * STAGES;   // MMAs of the stage finished
+  uint64_t* accum = bars + 3 * STAGES;   // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * BN;
+  const int nkb = (a.K + kGemmBK - 1) / kGemmBK;
+  constexpr int DEQ_WARP0 = 4;
+  constexpr int DEQ_WARPS = S::DEQ_THREADS / 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&bready[s], DEQ_WARPS);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&a.tmA);
+    prefetch_tmap(&a.tmP);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_acc = *tmem_slot;
+
+  // Weights and metadata do not depend on the previous kernel; X does.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      int issued = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % STAGES, r = kb / STAGES;
+        if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[s], S::A_BYTES + S::P_BYTES);
+        tma_load_2d(smem + s * S::STAGE_BYTES, &a.tmA, &full[s], kb * kGemmBK, m0);
+        tma_load_2d(p_ptr(s), &a.tmP, &full[s], kb * (kGemmBK / 2), n0);
+        ++issued;
+      }
+      // On abort, let copies already in flight land before the CTA leaves.
+      if (*abort_flag) {
+        for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
+          mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, ERR_TIMEOUT_TMA, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16_f32(kGemmBM, BN);
+      bool ok = true;
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int s = kb % STAGES, r = kb / STAGES;
+        ok = mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag) &&
+             mbar_wait(&bready[s], r & 1, ERR_TIMEOUT_PIPE, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t ad = desc_kmajor_sw128(a_addr(s));
+        const uint64_t bd = desc_kmajor_sw128(b_addr(s));
+#pragma unroll
+        for (int kk = 0; kk < kGemmBK / 16; ++kk)  // +32 bytes per K=16 step inside the swizzle atom
+          umma_bf16(tmem_acc, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), IDESC, (kb | kk) != 0);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accum);  // also on abort: completes when issued MMAs are done
+    }
+  } else if (warp >= DEQ_WARP0) {
+    // ---------------------------------------------------------- dequantize, then epilogue
+    const int t = threadIdx.x - DEQ_WARP0 * 32;  // weight row within the tile
+    const int n = min(n0 + t, a.N - 1);          // rows past N dequantize row N-1 (outputs masked)
+    const int ng = a.K >> a.log2g;
+    const uint32_t zw_stride = (ng + 7) >> 3;
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % STAGES, r = kb / STAGES;
+      // metadata first (independent of the stage)
+      uint32_t sc2 = 0, zoff2 = 0;
+      float sbv[4] = {0.f, 0.f, 0.f, 0.f};
+      if (FMT == 0) {
+        const int g = (kb * kGemmBK) >> a.log2g;
+        const float sc = __half2float(__ushort_as_half(__ldg(a.scales + int64_t(n) * ng + g)));
+        int z = 8;
+        if (a.zeros) z = (__ldg(a.zeros + int64_t(n) * zw_stride + (g >> 3)) >> (4 * (g & 7))) & 0xF;
+        sc2 = pack_bf16x2(sc, sc);
+        const uint32_t zb = 0x4300u | uint32_t(z);  // bf16(128 + z)
+        zoff2 = zb | (zb << 16);
+      } else {
+        const int nb = a.K >> 4;
+        const uint8_t* bs = a.bscale + int64_t(n) * nb + kb * 4;
+        const int rem = nb - kb * 4;  // K % 64 == 32 leaves two blocks in the last k-block
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sbv[q] = q < rem ? e4m3_decode_pos(__ldg(bs + q) & 0x7F) : 0.f;
+      }
+      if (!mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag)) { ok = false; break; }
+      const uint32_t prow = smem_u32(p_ptr(s)) + uint32_t(t * 32);
+      const uint4 q0 = ld_shared_v4(prow), q1 = ld_shared_v4(prow + 16);
+      const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      const uint32_t brow = b_addr(s);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint4 v = (FMT == 0) ? dequant_word_int4(words[j], zoff2, sc2) : dequant_word_nvfp4(words[j], sbv[j >> 1]);
+        if (a.inv_s) {
+          const int k = kb * kGemmBK + 8 * j;
+          if (k < a.K) {
+            const float4 i0 = __ldg(reinterpret_cast<const float4*>(a.inv_s + k));
+            const float4 i1 = __ldg(reinterpret_cast<const float4*>(a.inv_s + k) + 1);
+            v.x = bf16x2_mul(v.x, pack_bf16x2(i0.x, i0.y));
+            v.y = bf16x2_mul(v.y, pack_bf16x2(i0.z, i0.w));
+            v.z = bf16x2_mul(v.z, pack_bf16x2(i1.x, i1.y));
+            v.w = bf16x2_mul(v.w, pack_bf16x2(i1.z, i1.w));
+          }
+        }
+        st_shared_v4(brow + sw128_offset(t, j), v);
+      }
+      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bready[s]);
+    }
+    // ---------------------------------------------------------- epilogue
+    bool go = ok && mbar_wait(accum, 0, ERR_TIMEOUT_MMA, abort_flag);
+    go = __all_sync(0xffffffffu, go);  // tcgen05.ld below is warp-collective
+    if (go) {
+      tc_fence_after();
+      const int quarter = warp & 3;                // TMEM lanes 32*quarter .. +31
+      const int col0 = ((warp - DEQ_WARP0) >> 2) * 128;  // two warps per quarter when BN = 256
+      const int row = m0 + quarter * 32 + lane;
+      const float gmul = (FMT == 1) ? __ldg(a.gscale) : 1.0f;
+      const bool vec = (a.N % 8) == 0;
+      for (int c = col0; c < min(col0 + 128, BN); c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(c), v);
+        if (row < a.M) {
+          uint16_t* yrow = a.Y + int64_t(row) * a.N;
+          const int nb = n0 + c;
+          if (vec && nb + 32 <= a.N) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * gmul, __uint_as_float(v[8 * q + 1]) * gmul);
+              o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * gmul, __uint_as_float(v[8 * q + 3]) * gmul);
+              o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * gmul, __uint_as_float(v[8 * q + 5]) * gmul);
+              o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * gmul, __uint_as_float(v[8 * q + 7]) * gmul);
+              *reinterpret_cast<uint4*>(yrow + nb + 8 * q) = o;
+            }
+          } else {
+            for (int q = 0; q < 32; ++q)
+              if (nb + q < a.N) yrow[nb + q] = uint16_t(f32_to_bf16_bits(__uint_as_float(v[q]) * gmul));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_acc, BN);
+  }
+}
+
+}  // namespace wq

@@ -185,15 +185,13 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[r][m] = 0.f;
 
-  for (int it = it0; it < it1; ++it) {
+  // Packed weights of iteration `it` for the warp's R rows (zero past N or K).
+  auto load_w = [&](int it, uint4 (&wv)[R]) {
     const int kb = it * kGemvKPerIter + lane * 32;
-    if (kb >= K) continue;  // K % 32 == 0: a lane's 32 k are all in or all out
-    // packed weights of the R rows (issued first: the HBM stream)
-    uint4 wv[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int n = n0 + r;
-      if (n < N) {
+      if (n < N && it < it1 && kb < K) {
         if (FMT == FMT_INT4)
           wv[r] = ldg_stream_v4(static_cast<const uint32_t*>(a.wq) + int64_t(n) * (K / 8) + kb / 8);
         else
@@ -202,6 +200,23 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
         wv[r] = make_uint4(0, 0, 0, 0);
       }
     }
+  };
+
+  // Weights do not depend on the previous kernel in the stream: start
+  // streaming them, let the next kernel launch, and only then wait for the
+  // previous kernel's outputs (our activations) to become visible.
+  uint4 wnext[R];
+  load_w(it0, wnext);
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  for (int it = it0; it < it1; ++it) {
+    uint4 wv[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) wv[r] = wnext[r];
+    load_w(it + 1, wnext);  // register double buffering: next iteration in flight
+    const int kb = it * kGemvKPerIter + lane * 32;
+    if (kb >= K) continue;  // K % 32 == 0: a lane's 32 k are all in or all out
     // per-row metadata for this lane's 32 k
     float msc[R], mzf[R], md1[R];
 #pragma unroll

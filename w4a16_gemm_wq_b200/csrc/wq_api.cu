@@ -1,6 +1,7 @@
 // wq_api.cu -- host side of libwq: argument validation, launch configuration
 // and the extern "C" entry points declared in include/wq.h.  All kernels are
 // compiled into this one translation unit for sm_100a.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -9,6 +10,7 @@
 #include <algorithm>
 
 #include "../../include/wq.h"
+#include "gemm_tcgen05.cuh"
 #include "gemv.cuh"
 #include "quant.cuh"
 #include "wq_common.cuh"
@@ -85,13 +87,22 @@ int launch_gemv_mt(const wq::GemvArgs& a0, cudaStream_t st) {
   cfg.blockDim = dim3(wq::kGemvWarps * 32, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = splits;
-  attr[0].val.clusterDim.z = 1;
+  // Programmatic dependent launch: the kernel streams its weights before it
+  // waits (griddepcontrol.wait) for the previous kernel's outputs.
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (splits > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = splits;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = splits > 1 ? 1 : 0;
+  cfg.numAttrs = na;
   return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemv_kernel<FMT, MT>, a), "gemv launch");
 }
 
@@ -107,6 +118,79 @@ int log2i(int v) {
   while ((1 << r) < v) ++r;
   return r;
 }
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem` bytes, box [box_rows, box_cols].
+int make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, uint64_t rows, uint64_t cols,
+                 uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * uint64_t(elem)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(WQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return WQ_OK;
+}
+
+// ---------------------------------------------------------------- GEMM launch
+template <int FMT, int BN>
+int launch_gemm_bn(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaStream_t st) {
+  using S = wq::GemmShape<BN>;
+  if (int e = make_tmap_2d(&a.tmA, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(a.M), uint64_t(a.K),
+                           wq::kGemmBM, wq::kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B))
+    return e;
+  if (int e = make_tmap_2d(&a.tmP, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 2), BN,
+                           wq::kGemmBK / 2, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return e;
+  static bool attr_set = false;  // per instantiation; the value is the same on every device
+  if (!attr_set) {
+    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_tcgen05_kernel<FMT, BN>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES),
+                           "gemm smem attribute"))
+      return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((a.N + BN - 1) / BN, (a.M + wq::kGemmBM - 1) / wq::kGemmBM, 1);
+  cfg.blockDim = dim3(S::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = S::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemm_tcgen05_kernel<FMT, BN>, a), "gemm launch");
+}
+
+template <int FMT>
+int launch_gemm(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaStream_t st) {
+  const int64_t tiles256 = int64_t((a.N + 255) / 256) * ((a.M + wq::kGemmBM - 1) / wq::kGemmBM);
+  if (tiles256 >= 148) return launch_gemm_bn<FMT, 256>(a, X, packed, st);
+  return launch_gemm_bn<FMT, 128>(a, X, packed, st);
+}
+
+// Decode GEMV up to this many activation rows, tensor-core GEMM above.
+constexpr int64_t kGemvMaxM = 16;
 
 }  // namespace
 
@@ -259,6 +343,12 @@ int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uin
   } else {
     REQUIRE(!zeros, "zeros must be NULL for a symmetric (zero_point=0) pack");
   }
+  if (M > kGemvMaxM) {
+    wq::GemmArgs g = {};
+    g.scales = scales; g.zeros = zeros; g.inv_s = act_inv_s; g.Y = Y;
+    g.M = int(M); g.N = int(N); g.K = int(K); g.log2g = log2i(group_size);
+    return launch_gemm<wq::FMT_INT4>(g, X, qweight, as_stream(stream));
+  }
   wq::GemvArgs a = {};
   a.X = X; a.inv_s = act_inv_s; a.wq = qweight; a.scales = scales; a.zeros = zeros;
   a.Y = Y; a.M = int(M); a.N = int(N); a.K = int(K); a.log2g = log2i(group_size);
@@ -280,6 +370,12 @@ int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const ui
   REQUIRE_PTR(global_scale);
   REQUIRE_PTR(Y);
   REQUIRE_OPT_PTR(act_inv_s);
+  if (M > kGemvMaxM) {
+    wq::GemmArgs g = {};
+    g.bscale = bscale; g.gscale = global_scale; g.inv_s = act_inv_s; g.Y = Y;
+    g.M = int(M); g.N = int(N); g.K = int(K);
+    return launch_gemm<wq::FMT_NVFP4>(g, X, codes, as_stream(stream));
+  }
   wq::GemvArgs a = {};
   a.X = X; a.inv_s = act_inv_s; a.wq = codes; a.bscale = bscale; a.gscale = global_scale;
   a.Y = Y; a.M = int(M); a.N = int(N); a.K = int(K);
