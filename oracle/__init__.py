@@ -71,6 +71,8 @@ def _L():
         lib.oracle_activations_f64.argtypes = [P, I64, I64, P, P]
         lib.oracle_matmul_abT.restype = None
         lib.oracle_matmul_abT.argtypes = [P, I64, I64, P, I64, P]
+        lib.oracle_awq_delta.restype = I
+        lib.oracle_awq_delta.argtypes = [P, I64, I64, P, I, P]
         lib.oracle_awq_search.restype = I
         lib.oracle_awq_search.argtypes = [P, I64, I64, P, I64, P, P, I, I, P, P, P]
         lib.oracle_num_threads.restype = I
@@ -221,6 +223,23 @@ def linear(X, W_hat: np.ndarray, inv_s=None) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- AWQ
+def awq_delta(W, s, group_size: int) -> np.ndarray:
+    """Delta = W - dequant(Q(W s)) / s in fp64 [N, K]."""
+    w = as_bits16(W)
+    N, K = w.shape
+    out = np.empty((N, K), dtype=np.float64)
+    rc = _L().oracle_awq_delta(_ptr(w), N, K, _ptr(_f32(s)), group_size, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_awq_delta: invalid arguments")
+    return out
+
+
+def awq_mean_abs(X) -> np.ndarray:
+    """a_k = max(mean_t |X[t,k]|, 1e-4) in fp64 (the AWQ activation statistic)."""
+    x = activations_f64(X)
+    return np.maximum(np.abs(x).mean(axis=0), 1e-4)
+
+
 def awq_search(W, group_size: int, alphas, X=None, act_mean=None):
     """Returns (s fp32 [K], losses fp64 [n_alpha], best index)."""
     w = as_bits16(W)

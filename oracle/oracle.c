@@ -346,6 +346,22 @@ void oracle_matmul_abT(const double* A, int64_t M, int64_t K, const double* B, i
 /* AWQ grid search ([P1] "awq_apply.py"; [P4] section 7 AWQ)           */
 /* ------------------------------------------------------------------ */
 
+/* Delta = W - dequant(Q(W s)) / s in fp64 for one AWQ scale s (asymmetric
+ * INT4, group_size): the weight error the AWQ loss measures.  out is N x K. */
+int oracle_awq_delta(const uint16_t* W, int64_t N, int64_t K, const float* s, int group_size, double* out) {
+  if (N <= 0 || K <= 0 || K % group_size || !s) return ORACLE_ERR_ARG;
+  const int64_t ng = K / group_size, nzw = (ng + 7) / 8;
+  uint32_t* qw = malloc(sizeof(uint32_t) * N * (K / 8));
+  uint16_t* sc = malloc(sizeof(uint16_t) * N * ng);
+  uint32_t* zr = malloc(sizeof(uint32_t) * N * nzw);
+  oracle_quantize_int4(W, N, K, 4, group_size, 1, s, qw, sc, zr);
+  oracle_dequant_int4(qw, sc, zr, N, K, group_size, 1, NULL, 0, out);
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) out[n * K + k] = oracle_bf16_to_f64(W[n * K + k]) - out[n * K + k] / (double)s[k];
+  free(qw); free(sc); free(zr);
+  return ORACLE_OK;
+}
+
 /* For each alpha_i: s_k = fp32(a_k ^ alpha_i) with a_k = max(mean_t |X_tk|, 1e-4)
  * (or the given act_mean when X is NULL), W' = Q(W s) by the INT4 rule above
  * (asymmetric, group_size G), Delta = W - dequant(W') / s, and
@@ -363,13 +379,8 @@ int oracle_awq_search(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X
   if (N <= 0 || K <= 0 || n_alpha <= 0 || K % group_size) return ORACLE_ERR_ARG;
   if (X && T <= 0) return ORACLE_ERR_ARG;
   if (!X && !act_mean) return ORACLE_ERR_ARG;
-  const int64_t ng = K / group_size, nzw = (ng + 7) / 8;
   double* a = malloc(sizeof(double) * K);
   float* s = malloc(sizeof(float) * K);
-  uint32_t* qw = malloc(sizeof(uint32_t) * N * (K / 8));
-  uint16_t* sc = malloc(sizeof(uint16_t) * N * ng);
-  uint32_t* zr = malloc(sizeof(uint32_t) * N * nzw);
-  double* wh = malloc(sizeof(double) * N * K);
   double* delta = malloc(sizeof(double) * N * K);
   double* xd = X ? malloc(sizeof(double) * T * K) : NULL;
   double* y = X ? malloc(sizeof(double) * T * N) : NULL;
@@ -387,11 +398,7 @@ int oracle_awq_search(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X
   int best = 0;
   for (int i = 0; i < n_alpha; ++i) {
     for (int64_t k = 0; k < K; ++k) s[k] = (float)pow(a[k], (double)alphas[i]);
-    oracle_quantize_int4(W, N, K, 4, group_size, 1, s, qw, sc, zr);
-    oracle_dequant_int4(qw, sc, zr, N, K, group_size, 1, NULL, 0, wh);
-    for (int64_t n = 0; n < N; ++n)
-      for (int64_t k = 0; k < K; ++k)
-        delta[n * K + k] = oracle_bf16_to_f64(W[n * K + k]) - wh[n * K + k] / (double)s[k];
+    oracle_awq_delta(W, N, K, s, group_size, delta);
     double L = 0.0;
     if (X) {
       oracle_matmul_abT(xd, T, K, delta, N, y);
@@ -408,7 +415,7 @@ int oracle_awq_search(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X
   }
   for (int64_t k = 0; k < K; ++k) s_out[k] = (float)pow(a[k], (double)alphas[best]);
   *best_out = best;
-  free(a); free(s); free(qw); free(sc); free(zr); free(wh); free(delta); free(xd); free(y);
+  free(a); free(s); free(delta); free(xd); free(y);
   return ORACLE_OK;
 }
 

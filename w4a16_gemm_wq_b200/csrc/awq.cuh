@@ -1,0 +1,166 @@
+// awq.cuh -- AWQ grid search of the per-input-channel scale.
+//
+// "Lance-Quant", section "量化应用": awq_apply.py grid-searches an AWQ scale
+// equalization per layer before group-wise INT4 packing; section "校准阶段":
+// the calibration statistic is the mean absolute activation per input
+// channel.  "quantization primer", section 7 (AWQ): salient channels are
+// found from activation magnitudes and protected by scaling.
+//
+// For every alpha of the grid:
+//   s_k   = fp32(a_k ^ alpha),  a_k = max(mean_t |X[t,k]|, 1e-4)
+//   Delta = W - dequant(Q(W s)) / s           (asymmetric INT4, group G)
+//   L     = || X Delta^T ||_F^2               (tcgen05 GEMM, sum-of-squares epilogue)
+//   or, with no calibration tokens, L = sum_{n,k} (a_k Delta[n,k])^2.
+// Delta is stored as two bf16 planes (hi = bf16(Delta), lo = bf16(Delta - hi))
+// side by side, [N, 2K], so the loss GEMM X [T, K] x [hi | lo]^T over a
+// reduction of 2K keeps ~16 significant bits of Delta with bf16 tensor cores.
+// Every partial sum is written to its own slot and summed in a fixed order
+// in fp64: the losses are bit-reproducible run to run.
+#pragma once
+
+#include "quant.cuh"
+#include "wq_common.cuh"
+
+namespace wq {
+
+// a[k] = max(mean_t |X[t, k]|, 1e-4) (fp64), or max(act_mean[k], 1e-4).
+__global__ void __launch_bounds__(256) awq_act_mean_kernel(const uint16_t* __restrict__ X, int64_t T, int64_t K,
+                                                           const float* __restrict__ act_mean, double* __restrict__ a) {
+  const int64_t k = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+  double m;
+  if (X) {
+    double acc = 0.0;
+    for (int64_t t = 0; t < T; ++t) acc += fabs(double(bf16_bits_to_f32(X[t * K + k])));
+    m = acc / double(T);
+  } else {
+    m = double(act_mean[k]);
+  }
+  a[k] = m > 1e-4 ? m : 1e-4;
+}
+
+// s[k] = fp32(a[k] ^ alpha), alpha read from device memory.
+__global__ void __launch_bounds__(256) awq_scale_kernel(const double* __restrict__ a, const float* __restrict__ alpha,
+                                                        int64_t K, float* __restrict__ s) {
+  const int64_t k = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (k < K) s[k] = float(pow(a[k], double(*alpha)));
+}
+
+// Delta of one INT4 quantization round trip at scale s, same decisions as
+// quantize_int4_kernel (asymmetric).  grid = (ceil(K/2048), N).
+//   D != null: write Delta as bf16 hi at D[n, k] and lo at D[n, K + k].
+//   D == null: partials[cta] = sum over the CTA of (a_k * Delta[n,k])^2.
+template <int G>
+__global__ void __launch_bounds__(kQuantThreads) awq_delta_kernel(const uint16_t* __restrict__ W,
+                                                                  const float* __restrict__ s, int64_t N, int64_t K,
+                                                                  uint16_t* __restrict__ D,
+                                                                  const double* __restrict__ a,
+                                                                  double* __restrict__ partials) {
+  constexpr int LPG = G / 8;
+  const int64_t n = blockIdx.y;
+  const int64_t words = K / 8;
+  const int64_t u = int64_t(blockIdx.x) * kQuantThreads + threadIdx.x;
+  const bool active = u < words;
+  const int64_t k = u * 8;
+  float w[8], wp[8];
+  float mn = INFINITY, mx = -INFINITY;
+  if (active) {
+    load_wprime8(W, nullptr, K, n, k, w);
+    load_wprime8(W, s, K, n, k, wp);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      mn = fminf(mn, wp[j]);
+      mx = fmaxf(mx, wp[j]);
+    }
+  }
+#pragma unroll
+  for (int off = 1; off < LPG; off <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  float sc;
+  group_scale_f16(__fsub_rn(mx, mn), 15.0f, &sc);
+  const float z = fminf(fmaxf(rintf(__fdiv_rn(-mn, sc)), 0.0f), 15.0f);
+  double sq = 0.0;
+  if (active) {
+    float sv[8];
+    {
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + k));
+      const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + k + 4));
+      sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+      sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+    }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float q = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(wp[j], sc)), z), 0.0f), 15.0f);
+      const float deq = __fmul_rn(__fsub_rn(q, z), sc);        // exact: |q - z| <= 15, sc has 11 bits
+      const float dl = __fsub_rn(w[j], __fdiv_rn(deq, sv[j]));  // W - dequant / s
+      if (D) {
+        const uint32_t h = f32_to_bf16_bits(dl);
+        const uint32_t l = f32_to_bf16_bits(__fsub_rn(dl, bf16_bits_to_f32(h)));
+        if (j & 1) { hi[j >> 1] |= h << 16; lo[j >> 1] |= l << 16; }
+        else { hi[j >> 1] = h; lo[j >> 1] = l; }
+      } else {
+        const double v = a[k + j] * double(dl);
+        sq += v * v;
+      }
+    }
+    if (D) {
+      *reinterpret_cast<uint4*>(D + n * 2 * K + k) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      *reinterpret_cast<uint4*>(D + n * 2 * K + K + k) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+  }
+  if (!D) {
+    // fixed-order block reduction -> one partial per CTA
+    __shared__ double red[kQuantThreads / 32];
+#pragma unroll
+    for (int off = 16; off; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double t = 0.0;
+      for (int i = 0; i < kQuantThreads / 32; ++i) t += red[i];
+      partials[int64_t(blockIdx.y) * gridDim.x + blockIdx.x] = t;
+    }
+  }
+}
+
+// loss[i] = sum of partials[i*P .. i*P+P) (fp64, fixed order), best = first
+// argmin, s_out = fp32(a ^ alphas[best]).  One CTA.
+__global__ void __launch_bounds__(256) awq_finalize_kernel(const double* __restrict__ partials, int64_t P, int n_alpha,
+                                                           const double* __restrict__ a,
+                                                           const float* __restrict__ alphas, int64_t K,
+                                                           float* __restrict__ loss_out, int* __restrict__ best_out,
+                                                           float* __restrict__ s_out) {
+  __shared__ double red[256];
+  __shared__ double losses[1024];
+  __shared__ int best_sh;
+  for (int i = 0; i < n_alpha; ++i) {
+    double t = 0.0;
+    for (int64_t j = threadIdx.x; j < P; j += blockDim.x) t += partials[int64_t(i) * P + j];
+    red[threadIdx.x] = t;
+    __syncthreads();
+    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+      if (int(threadIdx.x) < w) red[threadIdx.x] += red[threadIdx.x + w];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+      losses[i] = red[0];
+      loss_out[i] = float(red[0]);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    int b = 0;
+    for (int i = 1; i < n_alpha; ++i)
+      if (losses[i] < losses[b]) b = i;
+    best_sh = b;
+    *best_out = b;
+  }
+  __syncthreads();
+  const double al = double(alphas[best_sh]);
+  for (int64_t k = threadIdx.x; k < K; k += blockDim.x) s_out[k] = float(pow(a[k], al));
+}
+
+}  // namespace wq

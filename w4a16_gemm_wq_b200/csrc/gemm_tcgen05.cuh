@@ -59,9 +59,14 @@ struct GemmArgs {
   const float* gscale;      // NVFP4 fp32 [1]
   const float* inv_s;       // fp32 [K] or null
   uint16_t* Y;              // bf16 [M, N]
-  int M, N, K;
+  double* sq_partials;      // FMT_BF16_SQ: one partial sum of squares per epilogue warp
+  int M, N, K;              // K: reduction length (for FMT_BF16_SQ the length of B's rows)
+  int a_kblocks;            // A k-block index wraps modulo this (FMT_BF16_SQ reuses X twice)
   int log2g;
 };
+
+// B operand modes of gemm_tcgen05_kernel.
+enum { GEMM_INT4 = 0, GEMM_NVFP4 = 1, GEMM_BF16_SQ = 2 };
 
 // ------------------------------------------------------------------ tcgen05 helpers
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
@@ -254,9 +259,15 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % STAGES, r = kb / STAGES;
         if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) break;
-        mbar_arrive_expect_tx(&full[s], S::A_BYTES + S::P_BYTES);
-        tma_load_2d(smem + s * S::STAGE_BYTES, &a.tmA, &full[s], kb * kGemmBK, m0);
-        tma_load_2d(p_ptr(s), &a.tmP, &full[s], kb * (kGemmBK / 2), n0);
+        if (FMT == GEMM_BF16_SQ) {
+          mbar_arrive_expect_tx(&full[s], S::A_BYTES + S::B_BYTES);
+          tma_load_2d(smem + s * S::STAGE_BYTES, &a.tmA, &full[s], (kb % a.a_kblocks) * kGemmBK, m0);
+          tma_load_2d(smem + s * S::STAGE_BYTES + S::A_BYTES, &a.tmP, &full[s], kb * kGemmBK, n0);
+        } else {
+          mbar_arrive_expect_tx(&full[s], S::A_BYTES + S::P_BYTES);
+          tma_load_2d(smem + s * S::STAGE_BYTES, &a.tmA, &full[s], kb * kGemmBK, m0);
+          tma_load_2d(p_ptr(s), &a.tmP, &full[s], kb * (kGemmBK / 2), n0);
+        }
         ++issued;
       }
       // On abort, let copies already in flight land before the CTA leaves.
@@ -273,7 +284,7 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
       for (int kb = 0; kb < nkb && ok; ++kb) {
         const int s = kb % STAGES, r = kb / STAGES;
         ok = mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag) &&
-             mbar_wait(&bready[s], r & 1, ERR_TIMEOUT_PIPE, abort_flag);
+             (FMT == GEMM_BF16_SQ || mbar_wait(&bready[s], r & 1, ERR_TIMEOUT_PIPE, abort_flag));
         if (!ok) break;
         tc_fence_after();
         const uint64_t ad = desc_kmajor_sw128(a_addr(s));
@@ -292,12 +303,12 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
     const int ng = a.K >> a.log2g;
     const uint32_t zw_stride = (ng + 7) >> 3;
     bool ok = true;
-    for (int kb = 0; kb < nkb; ++kb) {
+    for (int kb = 0; kb < (FMT == GEMM_BF16_SQ ? 0 : nkb); ++kb) {
       const int s = kb % STAGES, r = kb / STAGES;
       // metadata first (independent of the stage)
       uint32_t sc2 = 0, zoff2 = 0;
       float sbv[4] = {0.f, 0.f, 0.f, 0.f};
-      if (FMT == 0) {
+      if (FMT == GEMM_INT4) {
         const int g = (kb * kGemmBK) >> a.log2g;
         const float sc = __half2float(__ushort_as_half(__ldg(a.scales + int64_t(n) * ng + g)));
         int z = 8;
@@ -319,7 +330,7 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
       const uint32_t brow = b_addr(s);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        uint4 v = (FMT == 0) ? dequant_word_int4(words[j], zoff2, sc2) : dequant_word_nvfp4(words[j], sbv[j >> 1]);
+        uint4 v = (FMT == GEMM_INT4) ? dequant_word_int4(words[j], zoff2, sc2) : dequant_word_nvfp4(words[j], sbv[j >> 1]);
         if (a.inv_s) {
           const int k = kb * kGemmBK + 8 * j;
           if (k < a.K) {
@@ -345,11 +356,24 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
       const int quarter = warp & 3;                // TMEM lanes 32*quarter .. +31
       const int col0 = ((warp - DEQ_WARP0) >> 2) * 128;  // two warps per quarter when BN = 256
       const int row = m0 + quarter * 32 + lane;
-      const float gmul = (FMT == 1) ? __ldg(a.gscale) : 1.0f;
+      const float gmul = (FMT == GEMM_NVFP4) ? __ldg(a.gscale) : 1.0f;
       const bool vec = (a.N % 8) == 0;
+      double sq = 0.0;
       for (int c = col0; c < min(col0 + 128, BN); c += 32) {
         uint32_t v[32];
         tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(c), v);
+        if (FMT == GEMM_BF16_SQ) {
+          float part = 0.f;
+          if (row < a.M) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const float x = (n0 + c + q < a.N) ? __uint_as_float(v[q]) : 0.f;
+              part = fmaf(x, x, part);
+            }
+          }
+          sq += double(part);
+          continue;
+        }
         if (row < a.M) {
           uint16_t* yrow = a.Y + int64_t(row) * a.N;
           const int nb = n0 + c;
@@ -367,6 +391,15 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
             for (int q = 0; q < 32; ++q)
               if (nb + q < a.N) yrow[nb + q] = uint16_t(f32_to_bf16_bits(__uint_as_float(v[q]) * gmul));
           }
+        }
+      }
+      if (FMT == GEMM_BF16_SQ) {
+        // fixed-order warp reduction; one partial per (tile, epilogue warp)
+#pragma unroll
+        for (int off = 16; off; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        if (lane == 0) {
+          const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+          a.sq_partials[int64_t(tile) * DEQ_WARPS + (warp - DEQ_WARP0)] = sq;
         }
       }
     }

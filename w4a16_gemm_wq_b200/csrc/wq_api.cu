@@ -10,6 +10,7 @@
 #include <algorithm>
 
 #include "../../include/wq.h"
+#include "awq.cuh"
 #include "gemm_tcgen05.cuh"
 #include "gemv.cuh"
 #include "quant.cuh"
@@ -153,14 +154,8 @@ int make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int e
 
 // ---------------------------------------------------------------- GEMM launch
 template <int FMT, int BN>
-int launch_gemm_bn(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaStream_t st) {
+int launch_gemm_prepared(const wq::GemmArgs& a, cudaStream_t st) {
   using S = wq::GemmShape<BN>;
-  if (int e = make_tmap_2d(&a.tmA, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(a.M), uint64_t(a.K),
-                           wq::kGemmBM, wq::kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B))
-    return e;
-  if (int e = make_tmap_2d(&a.tmP, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 2), BN,
-                           wq::kGemmBK / 2, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return e;
   static bool attr_set = false;  // per instantiation; the value is the same on every device
   if (!attr_set) {
     if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_tcgen05_kernel<FMT, BN>,
@@ -182,11 +177,55 @@ int launch_gemm_bn(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaS
   return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemm_tcgen05_kernel<FMT, BN>, a), "gemm launch");
 }
 
+template <int FMT, int BN>
+int launch_gemm_bn(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaStream_t st) {
+  if (int e = make_tmap_2d(&a.tmA, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(a.M), uint64_t(a.K),
+                           wq::kGemmBM, wq::kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B))
+    return e;
+  if (int e = make_tmap_2d(&a.tmP, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 2), BN,
+                           wq::kGemmBK / 2, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return e;
+  return launch_gemm_prepared<FMT, BN>(a, st);
+}
+
+int gemm_bn(int64_t M, int64_t N);
+
 template <int FMT>
 int launch_gemm(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaStream_t st) {
-  const int64_t tiles256 = int64_t((a.N + 255) / 256) * ((a.M + wq::kGemmBM - 1) / wq::kGemmBM);
-  if (tiles256 >= 148) return launch_gemm_bn<FMT, 256>(a, X, packed, st);
+  if (gemm_bn(a.M, a.N) == 256) return launch_gemm_bn<FMT, 256>(a, X, packed, st);
   return launch_gemm_bn<FMT, 128>(a, X, packed, st);
+}
+
+int gemm_bn(int64_t M, int64_t N) {
+  const int64_t tiles256 = int64_t((N + 255) / 256) * ((M + wq::kGemmBM - 1) / wq::kGemmBM);
+  return tiles256 >= 148 ? 256 : 128;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Workspace of awq_search_scale: a (fp64 [K]), s (fp32 [K]), loss partials
+// (fp64 [n_alpha, P]) and, with calibration tokens, Delta (bf16 [N, 2K]).
+struct AwqLayout {
+  size_t off_a, off_s, off_p, off_d, total;
+  int64_t P;
+  int bn;
+};
+
+AwqLayout awq_layout(int64_t N, int64_t K, int64_t T, bool has_x, int n_alpha) {
+  AwqLayout L = {};
+  if (has_x) {
+    L.bn = gemm_bn(T, N);
+    L.P = ((N + L.bn - 1) / L.bn) * ((T + wq::kGemmBM - 1) / wq::kGemmBM) * (L.bn / 32);
+  } else {
+    L.bn = 0;
+    L.P = ((K / 8 + wq::kQuantThreads - 1) / wq::kQuantThreads) * N;
+  }
+  L.off_a = 0;
+  L.off_s = align256(L.off_a + size_t(K) * 8);
+  L.off_p = align256(L.off_s + size_t(K) * 4);
+  L.off_d = align256(L.off_p + size_t(n_alpha) * size_t(L.P) * 8);
+  L.total = has_x ? align256(L.off_d + size_t(N) * size_t(2 * K) * 2) : L.off_d;
+  return L;
 }
 
 // Decode GEMV up to this many activation rows, tensor-core GEMM above.
@@ -241,10 +280,10 @@ int awq_search_workspace_size(int64_t N, int64_t K, int64_t T, int n_alpha, int 
   REQUIRE(bytes, "bytes must not be NULL");
   if (int e = check_shape(N, K)) return e;
   if (int e = check_group(group_size, K)) return e;
-  (void)T;
-  (void)n_alpha;
-  *bytes = 0;
-  return fail(WQ_ERR_UNSUPPORTED, "awq_search_scale is not available in this build");
+  REQUIRE(T >= 0, "T must not be negative");
+  REQUIRE(n_alpha > 0 && n_alpha <= 1024, "n_alpha must be in 1..1024");
+  *bytes = awq_layout(N, K, T, T > 0, n_alpha).total;
+  return WQ_OK;
 }
 
 int wq_quantize_int4(const uint16_t* W, int64_t N, int64_t K, int bits, int group_size, int zero_point,
@@ -320,8 +359,47 @@ int awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X,
   REQUIRE_PTR(s_out);
   REQUIRE_PTR(loss_out);
   REQUIRE_PTR(best_idx);
-  (void)ws; (void)ws_bytes; (void)stream;
-  return fail(WQ_ERR_UNSUPPORTED, "awq_search_scale is not available in this build");
+  const AwqLayout L = awq_layout(N, K, X ? T : 0, X != nullptr, n_alpha);
+  REQUIRE(ws && ws_bytes >= L.total, "workspace too small: need %zu bytes (awq_search_workspace_size)", L.total);
+  REQUIRE_PTR(ws);
+  cudaStream_t st = as_stream(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  double* a = reinterpret_cast<double*>(wsb + L.off_a);
+  float* s = reinterpret_cast<float*>(wsb + L.off_s);
+  double* partials = reinterpret_cast<double*>(wsb + L.off_p);
+  uint16_t* D = X ? reinterpret_cast<uint16_t*>(wsb + L.off_d) : nullptr;
+
+  wq::awq_act_mean_kernel<<<unsigned((K + 255) / 256), 256, 0, st>>>(X, T, K, act_mean, a);
+  if (int e = launched("awq_act_mean launch")) return e;
+  wq::GemmArgs g = {};
+  if (X) {
+    g.M = int(T); g.N = int(N); g.K = int(2 * K); g.a_kblocks = int(K / wq::kGemmBK);
+    if (int e = make_tmap_2d(&g.tmA, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(T), uint64_t(K), wq::kGemmBM,
+                             wq::kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B))
+      return e;
+    if (int e = make_tmap_2d(&g.tmP, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(N), uint64_t(2 * K), L.bn,
+                             wq::kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B))
+      return e;
+  }
+  const dim3 dgrid(unsigned((K / 8 + wq::kQuantThreads - 1) / wq::kQuantThreads), unsigned(N));
+  for (int i = 0; i < n_alpha; ++i) {
+    wq::awq_scale_kernel<<<unsigned((K + 255) / 256), 256, 0, st>>>(a, alphas + i, K, s);
+    if (int e = launched("awq_scale launch")) return e;
+    double* part_i = partials + int64_t(i) * L.P;
+    if (group_size == 64)
+      wq::awq_delta_kernel<64><<<dgrid, wq::kQuantThreads, 0, st>>>(W, s, N, K, D, a, part_i);
+    else
+      wq::awq_delta_kernel<128><<<dgrid, wq::kQuantThreads, 0, st>>>(W, s, N, K, D, a, part_i);
+    if (int e = launched("awq_delta launch")) return e;
+    if (X) {
+      g.sq_partials = part_i;
+      const int e = (L.bn == 256) ? launch_gemm_prepared<wq::GEMM_BF16_SQ, 256>(g, st)
+                                  : launch_gemm_prepared<wq::GEMM_BF16_SQ, 128>(g, st);
+      if (e) return e;
+    }
+  }
+  wq::awq_finalize_kernel<<<1, 256, 0, st>>>(partials, L.P, n_alpha, a, alphas, K, loss_out, best_idx, s_out);
+  return launched("awq_finalize launch");
 }
 
 int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* qweight,
