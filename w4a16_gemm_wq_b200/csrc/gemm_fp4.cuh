@@ -1,0 +1,245 @@
+// gemm_fp4.cuh -- NVFP4 W4A4 GEMM on the block-scaled FP4 tensor cores
+// (tcgen05.mma kind::mxf4nvf4, one E4M3 scale per 16 elements).
+//
+// "OmniQuant" section 4.2 (W4A4: weights and activations both 4-bit);
+// "Lance-Quant" section "量化应用" (NVFP4 = E2M1 codes + E4M3 scale per 16,
+// for Blackwell tensor cores).  The activations were quantized to NVFP4 along
+// K just before (same rule as the weight pack, own per-tensor scale g_x):
+//   Y[m, n] = g_x g_w sum_b sx[m,b] sw[n,b] sum_{k in b} e2m1(xq[m,k]) e2m1(wq[n,k])
+// which is exactly what the block-scaled MMA computes (fp32 accumulation);
+// the two per-tensor scales multiply the accumulator in the epilogue.
+//
+// One CTA = one 128 x BN output tile; k-blocks of 256 elements (128 bytes of
+// packed E2M1 per row = one 128-byte swizzle atom), STAGES deep:
+//   warp 0      TMA: packed X tile [128 x 128 B] and W tile [BN x 128 B]
+//   warp 1      TMEM allocation (512 columns) and the tcgen05.mma issuer
+//               (4 MMAs of K = 64 per k-block)
+//   warps 4..11 copy the stage's E4M3 scales into tensor memory with
+//               tcgen05.st (warps 4-7: X scales, 8-11: W scales), then run the
+//               epilogue (tcgen05.ld, x g_x g_w, bf16 store).
+// Scale-factor placement in tensor memory: the four scales (4 bytes) of row r
+// for one K = 64 step form one 32-bit word at column (r / 32) and lane
+// (r % 32) of every 32-lane subpartition.
+#pragma once
+
+#include "gemm_tcgen05.cuh"
+
+namespace wq {
+
+constexpr int kFp4BK = 256;  // elements per k-block
+
+template <int BN>
+struct Fp4Shape {
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = kGemmBM * kFp4BK / 2;  // 16 KB
+  static constexpr int B_BYTES = BN * kFp4BK / 2;       // 32 KB at BN = 256
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int THREADS = 384;
+  static constexpr int SFA_COLS = 4 * 4;         // 4 K-steps x 4 row blocks of 32
+  static constexpr int SFB_COLS = 4 * (BN / 32);
+  static constexpr int SF_STAGE_COLS = SFA_COLS + SFB_COLS;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(256 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+};
+
+struct Fp4Args {
+  CUtensorMap tmA;        // X codes u8 [M, K/2], box {128 B, 128}, 128B swizzle
+  CUtensorMap tmB;        // W codes u8 [N, K/2], box {128 B, BN}, 128B swizzle
+  const uint8_t* sfa;     // X e4m3 [M, K/16]
+  const uint8_t* sfb;     // W e4m3 [N, K/16]
+  const float* gx;        // fp32 [1]
+  const float* gw;        // fp32 [1]
+  uint16_t* Y;            // bf16 [M, N]
+  int M, N, K;            // K % 64 == 0
+};
+
+// Instruction descriptor: E2M1 x E2M1 with E4M3 block scales, fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);  // scale format 0 = E4M3
+}
+
+__device__ __forceinline__ void umma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// Four scale bytes (one K = 64 step) of row `row` at k-step `ks`, zero outside.
+__device__ __forceinline__ uint32_t sf_word(const uint8_t* __restrict__ sf, int row, int rows, int ks, int ksteps,
+                                            int stride) {
+  if (row >= rows || ks >= ksteps) return 0u;
+  return __ldg(reinterpret_cast<const uint32_t*>(sf + int64_t(row) * stride) + ks);
+}
+
+template <int BN>
+__global__ void __launch_bounds__(Fp4Shape<BN>::THREADS, 1) gemm_fp4_kernel(const __grid_constant__ Fp4Args a) {
+  using S = Fp4Shape<BN>;
+  constexpr int STAGES = S::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* sfready = bars + STAGES;
+  uint64_t* empty = bars + 2 * STAGES;
+  uint64_t* accum = bars + 3 * STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * BN;
+  const int nkb = (a.K + kFp4BK - 1) / kFp4BK;
+  const int ksteps = a.K / 64;     // valid K = 64 steps
+  const int sf_stride = a.K / 16;  // bytes per row of the scale arrays
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&sfready[s], 8);  // the 8 scale-copy warps
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&a.tmA);
+    prefetch_tmap(&a.tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_acc = tmem;
+  auto sfa_col = [&](int s) { return uint32_t(256 + s * S::SF_STAGE_COLS); };
+  auto sfb_col = [&](int s) { return uint32_t(256 + s * S::SF_STAGE_COLS + S::SFA_COLS); };
+
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (warp == 0) {
+    if (lane == 0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      int issued = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % STAGES, r = kb / STAGES;
+        if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) break;
+        mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+        tma_load_2d(smem + s * S::STAGE_BYTES, &a.tmA, &full[s], kb * (kFp4BK / 2), m0);
+        tma_load_2d(smem + s * S::STAGE_BYTES + S::A_BYTES, &a.tmB, &full[s], kb * (kFp4BK / 2), n0);
+        ++issued;
+      }
+      if (*abort_flag) {
+        for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
+          mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, ERR_TIMEOUT_TMA, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_nvf4(kGemmBM, BN);
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = kb % STAGES, r = kb / STAGES;
+        if (!mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag)) break;
+        if (!mbar_wait(&sfready[s], r & 1, ERR_TIMEOUT_PIPE, abort_flag)) break;
+        tc_fence_after();
+        const uint64_t ad = desc_kmajor_sw128(sbase + uint32_t(s * S::STAGE_BYTES));
+        const uint64_t bd = desc_kmajor_sw128(sbase + uint32_t(s * S::STAGE_BYTES + S::A_BYTES));
+#pragma unroll
+        for (int t = 0; t < 4; ++t)  // K = 64 per MMA: +32 bytes inside the swizzle atom
+          umma_nvf4(tmem_acc, ad + uint64_t(2 * t), bd + uint64_t(2 * t), IDESC, tmem + sfa_col(s) + 4 * t,
+                    tmem + sfb_col(s) + (BN / 32) * t, (kb | t) != 0);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accum);
+    }
+  } else if (warp >= 4) {
+    const int quarter = warp & 3;
+    const bool is_b = warp >= 8;
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    bool ok = true;
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % STAGES, r = kb / STAGES;
+      if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) { ok = false; break; }
+      if (!is_b) {
+        uint32_t v[16];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) v[4 * t + c] = sf_word(a.sfa, m0 + lane + 32 * c, a.M, 4 * kb + t, ksteps, sf_stride);
+        tmem_st16(tmem + lane_base + sfa_col(s), v);
+      } else {
+#pragma unroll
+        for (int h = 0; h < S::SFB_COLS / 16; ++h) {  // 16 columns per store
+          uint32_t v[16];
+#pragma unroll
+          for (int t2 = 0; t2 < 16; ++t2) {
+            const int col = 16 * h + t2;            // column within the stage's SFB block
+            const int t = col / (BN / 32), c = col % (BN / 32);
+            v[t2] = sf_word(a.sfb, n0 + lane + 32 * c, a.N, 4 * kb + t, ksteps, sf_stride);
+          }
+          tmem_st16(tmem + lane_base + sfb_col(s) + 16 * h, v);
+        }
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sfready[s]);
+    }
+    // ---------------------------------------------------------- epilogue
+    bool go = ok && mbar_wait(accum, 0, ERR_TIMEOUT_MMA, abort_flag);
+    go = __all_sync(0xffffffffu, go);
+    if (go) {
+      tc_fence_after();
+      const int col0 = is_b ? 128 : 0;
+      const int row = m0 + quarter * 32 + lane;
+      const float gmul = __ldg(a.gx) * __ldg(a.gw);
+      const bool vec = (a.N % 8) == 0;
+      for (int c = col0; c < min(col0 + 128, BN); c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem_acc + lane_base + uint32_t(c), v);
+        if (row < a.M) {
+          uint16_t* yrow = a.Y + int64_t(row) * a.N;
+          const int nb = n0 + c;
+          if (vec && nb + 32 <= a.N) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * gmul, __uint_as_float(v[8 * q + 1]) * gmul);
+              o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * gmul, __uint_as_float(v[8 * q + 3]) * gmul);
+              o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * gmul, __uint_as_float(v[8 * q + 5]) * gmul);
+              o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * gmul, __uint_as_float(v[8 * q + 7]) * gmul);
+              *reinterpret_cast<uint4*>(yrow + nb + 8 * q) = o;
+            }
+          } else {
+            for (int q = 0; q < 32; ++q)
+              if (nb + q < a.N) yrow[nb + q] = uint16_t(f32_to_bf16_bits(__uint_as_float(v[q]) * gmul));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, S::TMEM_COLS);
+  }
+}
+
+}  // namespace wq

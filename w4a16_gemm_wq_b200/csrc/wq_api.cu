@@ -11,6 +11,7 @@
 
 #include "../../include/wq.h"
 #include "awq.cuh"
+#include "gemm_fp4.cuh"
 #include "gemm_tcgen05.cuh"
 #include "gemv.cuh"
 #include "quant.cuh"
@@ -228,6 +229,68 @@ AwqLayout awq_layout(int64_t N, int64_t K, int64_t T, bool has_x, int n_alpha) {
   return L;
 }
 
+// Workspace of the W4A4 path: X as NVFP4 (codes [M, K/2], E4M3 scales
+// [M, K/16]) and its per-tensor scale g_x.
+struct W4A4Layout {
+  size_t off_codes, off_sf, off_g, total;
+};
+
+W4A4Layout w4a4_layout(int64_t M, int64_t K) {
+  W4A4Layout L = {};
+  L.off_codes = 0;
+  L.off_sf = align256(size_t(M) * size_t(K / 2));
+  L.off_g = align256(L.off_sf + size_t(M) * size_t(K / 16));
+  L.total = L.off_g + 256;
+  return L;
+}
+
+template <int BN>
+int launch_fp4_bn(wq::Fp4Args& a, const uint8_t* xcodes, const uint8_t* wcodes, cudaStream_t st) {
+  using S = wq::Fp4Shape<BN>;
+  if (int e = make_tmap_2d(&a.tmA, xcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.M), uint64_t(a.K / 2),
+                           wq::kGemmBM, wq::kFp4BK / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+    return e;
+  if (int e = make_tmap_2d(&a.tmB, wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 2), BN,
+                           wq::kFp4BK / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+    return e;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_fp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                S::SMEM_BYTES),
+                           "fp4 gemm smem attribute"))
+      return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((a.N + BN - 1) / BN, (a.M + wq::kGemmBM - 1) / wq::kGemmBM, 1);
+  cfg.blockDim = dim3(S::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = S::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemm_fp4_kernel<BN>, a), "fp4 gemm launch");
+}
+
+// NVFP4 quantization of a bf16 [R, C] tensor (optionally times s per column)
+// into codes / scales / g: the three stream-ordered passes of wq_quantize_nvfp4.
+int nvfp4_quantize_launch(const uint16_t* A, int64_t R, int64_t C, const float* s, uint8_t* codes, uint8_t* bscale,
+                          float* g, cudaStream_t st) {
+  if (int e = cuda_check(cudaMemsetAsync(g, 0, sizeof(float), st), "memset")) return e;
+  const int64_t words = R * C / 8;
+  const int amax_blocks = int(std::min<int64_t>((words + 255) / 256, 148 * 8));
+  wq::nvfp4_amax_kernel<<<amax_blocks, 256, 0, st>>>(A, s, R, C, g);
+  if (int e = launched("nvfp4_amax launch")) return e;
+  const int64_t nblk = R * C / 16;
+  const int pack_blocks = int(std::min<int64_t>((nblk + 255) / 256, 148 * 16));
+  wq::nvfp4_pack_kernel<<<pack_blocks, 256, 0, st>>>(A, s, R, C, g, codes, bscale);
+  if (int e = launched("nvfp4_pack launch")) return e;
+  wq::nvfp4_finalize_kernel<<<1, 1, 0, st>>>(g);
+  return launched("nvfp4_finalize launch");
+}
+
 // Decode GEMV up to this many activation rows, tensor-core GEMM above.
 constexpr int64_t kGemvMaxM = 16;
 
@@ -271,8 +334,9 @@ int wq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int format, int ac
   REQUIRE(M > 0, "M must be positive");
   if (int e = check_shape(N, K)) return e;
   REQUIRE(format == WQ_FMT_INT4 || format == WQ_FMT_NVFP4, "unknown format %d", format);
-  *bytes = 0;
-  (void)act_fp4;
+  REQUIRE(act_fp4 == 0 || act_fp4 == 1, "act_fp4 must be 0 or 1");
+  REQUIRE(!act_fp4 || format == WQ_FMT_NVFP4, "act_fp4 needs the NVFP4 format");
+  *bytes = act_fp4 ? w4a4_layout(M, K).total : 0;
   return WQ_OK;
 }
 
@@ -325,20 +389,9 @@ int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scal
   REQUIRE_PTR(bscale);
   REQUIRE_PTR(global_scale);
   REQUIRE_OPT_PTR(scale_s);
-  cudaStream_t st = as_stream(stream);
   // global_scale first accumulates amax, then the pack pass reads it, then it
   // is replaced by g: three stream-ordered steps, no scratch memory.
-  if (int e = cuda_check(cudaMemsetAsync(global_scale, 0, sizeof(float), st), "memset")) return e;
-  const int64_t words = N * K / 8;
-  const int amax_blocks = int(std::min<int64_t>((words + 255) / 256, 148 * 8));
-  wq::nvfp4_amax_kernel<<<amax_blocks, 256, 0, st>>>(W, scale_s, N, K, global_scale);
-  if (int e = launched("nvfp4_amax launch")) return e;
-  const int64_t nblk = N * K / 16;
-  const int pack_blocks = int(std::min<int64_t>((nblk + 255) / 256, 148 * 16));
-  wq::nvfp4_pack_kernel<<<pack_blocks, 256, 0, st>>>(W, scale_s, N, K, global_scale, codes, bscale);
-  if (int e = launched("nvfp4_pack launch")) return e;
-  wq::nvfp4_finalize_kernel<<<1, 1, 0, st>>>(global_scale);
-  return launched("nvfp4_finalize launch");
+  return nvfp4_quantize_launch(W, N, K, scale_s, codes, bscale, global_scale, as_stream(stream));
 }
 
 int awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t T, const float* act_mean,
@@ -441,13 +494,28 @@ int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const ui
   REQUIRE(M > 0 && M <= (int64_t(1) << 30), "M must be positive");
   if (int e = check_shape(N, K)) return e;
   REQUIRE(act_fp4 == 0 || act_fp4 == 1, "act_fp4 must be 0 or 1");
-  if (act_fp4) return fail(WQ_ERR_UNSUPPORTED, "W4A4 (act_fp4=1) is not available in this build");
   REQUIRE_PTR(X);
   REQUIRE_PTR(codes);
   REQUIRE_PTR(bscale);
   REQUIRE_PTR(global_scale);
   REQUIRE_PTR(Y);
   REQUIRE_OPT_PTR(act_inv_s);
+  if (act_fp4) {
+    REQUIRE(K % 64 == 0, "W4A4 needs K %% 64 == 0 (got %lld)", (long long)K);
+    const W4A4Layout L = w4a4_layout(M, K);
+    REQUIRE(ws && ws_bytes >= L.total, "workspace too small: need %zu bytes (wq_linear_workspace_size)", L.total);
+    REQUIRE_PTR(ws);
+    cudaStream_t st = as_stream(stream);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    uint8_t* xcodes = wsb + L.off_codes;
+    uint8_t* xsf = wsb + L.off_sf;
+    float* gx = reinterpret_cast<float*>(wsb + L.off_g);
+    if (int e = nvfp4_quantize_launch(X, M, K, act_inv_s, xcodes, xsf, gx, st)) return e;
+    wq::Fp4Args f = {};
+    f.sfa = xsf; f.sfb = bscale; f.gx = gx; f.gw = global_scale; f.Y = Y;
+    f.M = int(M); f.N = int(N); f.K = int(K);
+    return gemm_bn(M, N) == 256 ? launch_fp4_bn<256>(f, xcodes, codes, st) : launch_fp4_bn<128>(f, xcodes, codes, st);
+  }
   if (M > kGemvMaxM) {
     wq::GemmArgs g = {};
     g.bscale = bscale; g.gscale = global_scale; g.inv_s = act_inv_s; g.Y = Y;
