@@ -23,7 +23,8 @@
  *  - bf16 and fp16 values travel as their 16-bit patterns (uint16_t).
  *  - All data pointers are DEVICE pointers owned by the caller; the library
  *    allocates no memory and keeps no state except one device error word
- *    per loaded GPU (see wq_device_error).
+ *    per loaded GPU (see wq_device_error) and the fixed scratch array of
+ *    wq_linear_nvfp4_w4a4_noalloc.
  *  - `stream` is a cudaStream_t (0 = legacy default stream).  Every call is
  *    asynchronous on that stream; validation happens on the host before any
  *    launch, so an error return means nothing was launched.
@@ -173,6 +174,27 @@ int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uin
 int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
                     const uint8_t* bscale, const float* global_scale, int act_fp4,
                     const float* act_inv_s, uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* wq_linear_nvfp4_w4a4_noalloc -- the W4A4 product of wq_linear_nvfp4
+ * (act_fp4 = 1) for callers that cannot allocate device memory when they
+ * call, and so cannot hand over a workspace: for example a runtime that
+ * plans every device buffer up front and forbids allocation afterwards, or
+ * code running where no device allocator is reachable.  The pages have no
+ * counterpart of this entry point; it exists only for such callers.
+ *   Arguments as for wq_linear_nvfp4 with act_fp4 = 1, minus the workspace.
+ *   The NVFP4 pack of X is kept in a scratch array inside the library
+ *   (8 MiB per GPU that loads the library, held until the process exits).
+ *   The pack needs M*K/2 + M*K/16 bytes plus alignment; larger problems are
+ *   rejected with WQ_ERR_ARG (use wq_linear_nvfp4 with a workspace then).
+ *   The call allocates nothing.  Its first call on a GPU looks up the
+ *   scratch array's device address there; make that first call before any
+ *   CUDA graph capture.  All calls on a GPU share the one array: calls whose
+ *   execution overlaps on the GPU (different streams without ordering) race
+ *   on it and give undefined results. */
+int wq_linear_nvfp4_w4a4_noalloc(const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                                 const uint8_t* codes, const uint8_t* bscale,
+                                 const float* global_scale, const float* act_inv_s, uint16_t* Y,
+                                 void* stream);
 
 /* Synchronizes `stream`, then reads and clears the device error word of the
  * current GPU.  WQ_OK if no kernel reported a problem since the last call,

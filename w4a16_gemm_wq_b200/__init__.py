@@ -40,6 +40,7 @@ SIGNATURES = {
     "awq_search_scale": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "wq_linear_int4": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "wq_linear_nvfp4": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]),
+    "wq_linear_nvfp4_w4a4_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P]),
     "wq_device_error": (_I, [_P]),
 }
 
@@ -248,6 +249,23 @@ def wq_linear_nvfp4(X: torch.Tensor, p: PackedNVFP4, act_fp4: int = 0, act_inv_s
     _check(lib.wq_linear_nvfp4(_ptr(X), M, p.N, K, _ptr(p.codes), _ptr(p.bscale), _ptr(p.global_scale), act_fp4,
                                _ptr(s), _ptr(Y), _ptr(ws), 0 if ws is None else ws.numel(), _stream()),
            "wq_linear_nvfp4")
+    return Y
+
+
+def wq_linear_nvfp4_w4a4_noalloc(X: torch.Tensor, p: PackedNVFP4, act_inv_s=None,
+                                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """W4A4 product without a workspace: the library's fixed scratch holds the
+    NVFP4 pack of X (for callers that cannot allocate at call time)."""
+    _dev(X, "X", torch.bfloat16)
+    M, K = X.shape
+    if K != p.K:
+        raise ValueError(f"X has K={K}, the pack K={p.K}")
+    Y = out if out is not None else torch.empty((M, p.N), dtype=torch.bfloat16, device=X.device)
+    _dev(Y, "out", torch.bfloat16, (M, p.N))
+    s = _opt_f32(act_inv_s, "act_inv_s", K)
+    _check(load().wq_linear_nvfp4_w4a4_noalloc(_ptr(X), M, p.N, K, _ptr(p.codes), _ptr(p.bscale),
+                                               _ptr(p.global_scale), _ptr(s), _ptr(Y), _stream()),
+           "wq_linear_nvfp4_w4a4_noalloc")
     return Y
 
 

@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "../../include/wq.h"
 #include "awq.cuh"
@@ -294,6 +295,35 @@ int nvfp4_quantize_launch(const uint16_t* A, int64_t R, int64_t C, const float* 
 // Decode GEMV up to this many activation rows, tensor-core GEMM above.
 constexpr int64_t kGemvMaxM = 16;
 
+// ---------------------------------------------------------------- fixed scratch
+// Scratch memory of wq_linear_nvfp4_w4a4_noalloc, owned by the library: the
+// NVFP4 pack of X (codes | E4M3 scales | g_x, laid out as w4a4_layout) lives
+// in this array instead of a caller-provided workspace.  Every GPU that loads
+// the library holds these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per GPU
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current GPU.  In host code the
+// array's name only stands for the symbol, so the address is looked up once
+// per device (cudaGetSymbolAddress, with that device current) and cached.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (int e = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return e;
+  if (dev < 0 || dev >= kMaxDevices) return fail(WQ_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (int e = cuda_check(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress")) return e;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return WQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -526,6 +556,38 @@ int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const ui
   a.X = X; a.inv_s = act_inv_s; a.wq = codes; a.bscale = bscale; a.gscale = global_scale;
   a.Y = Y; a.M = int(M); a.N = int(N); a.K = int(K);
   return launch_gemv<wq::FMT_NVFP4>(a, as_stream(stream));
+}
+
+int wq_linear_nvfp4_w4a4_noalloc(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
+                                  const uint8_t* bscale, const float* global_scale, const float* act_inv_s,
+                                  uint16_t* Y, void* stream) {
+  REQUIRE(M > 0 && M <= (int64_t(1) << 30), "M must be positive");
+  if (int e = check_shape(N, K)) return e;
+  REQUIRE(K % 64 == 0, "W4A4 needs K %% 64 == 0 (got %lld)", (long long)K);
+  REQUIRE_PTR(X);
+  REQUIRE_PTR(codes);
+  REQUIRE_PTR(bscale);
+  REQUIRE_PTR(global_scale);
+  REQUIRE_PTR(Y);
+  REQUIRE_OPT_PTR(act_inv_s);
+  const W4A4Layout L = w4a4_layout(M, K);
+  REQUIRE(L.total <= kNoAllocScratchBytes,
+          "M x K = %lld x %lld needs %zu bytes of scratch, more than the fixed %zu bytes of this entry point; "
+          "use wq_linear_nvfp4 with a workspace",
+          (long long)M, (long long)K, L.total, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if (int e = noalloc_scratch(&scratch)) return e;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(scratch);
+  uint8_t* xcodes = wsb + L.off_codes;
+  uint8_t* xsf = wsb + L.off_sf;
+  float* gx = reinterpret_cast<float*>(wsb + L.off_g);
+  // nvfp4_quantize_launch zeroes g_x (the amax accumulator) before using it
+  if (int e = nvfp4_quantize_launch(X, M, K, act_inv_s, xcodes, xsf, gx, st)) return e;
+  wq::Fp4Args f = {};
+  f.sfa = xsf; f.sfb = bscale; f.gx = gx; f.gw = global_scale; f.Y = Y;
+  f.M = int(M); f.N = int(N); f.K = int(K);
+  return gemm_bn(M, N) == 256 ? launch_fp4_bn<256>(f, xcodes, codes, st) : launch_fp4_bn<128>(f, xcodes, codes, st);
 }
 
 int wq_device_error(void* stream) {
