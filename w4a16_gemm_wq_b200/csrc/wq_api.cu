@@ -10,7 +10,7 @@
 #include <algorithm>
 #include <mutex>
 
-#include "../../include/wq.h"
+#include "wq.h"
 #include "awq.cuh"
 #include "gemm_fp4.cuh"
 #include "gemm_tcgen05.cuh"
