@@ -39,9 +39,15 @@ def load_peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
-                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
-    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+        pk = dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                  bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
+    else:
+        pk = dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+    # dense FP4 is not measured on this machine: the measured bf16 figure times the
+    # nominal dense FP4 / bf16 ratio (9 / 2.25 PFLOP/s = 4)
+    pk["fp4"] = 4.0 * pk["bf16"]
+    pk["fp4_sustained"] = 4.0 * pk["bf16_sustained"]
+    return pk
 
 
 class ClockSampler:
@@ -101,11 +107,7 @@ class ClockSampler:
                 "reasons": sorted(seen), "samples": len(rows)}
 
 
-def dist_env():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return ws, rank, local
+from w4a16_gemm_wq_b200.dist import dist_env, max_over_ranks  # noqa: E402
 
 
 # ---------------------------------------------------------------- our arm
@@ -192,11 +194,7 @@ def run_ours(args):
             graphs[(args.warmup + i) % len(graphs)].replay()
         stop.record()
         torch.cuda.synchronize()
-    ms = start.elapsed_time(stop)
-    if pg:
-        t = torch.tensor([ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = t.item()
+    ms = max_over_ranks([start.elapsed_time(stop)], device=dev)[0]
 
     # per-kind breakdown: a graph of `reps` launches of one kind, rotating copies
     detail = {}
@@ -254,11 +252,7 @@ def run_ours(args):
         egraphs[(args.warmup + i) % len(egraphs)].replay()
     e2.record()
     torch.cuda.synchronize()
-    ms2 = s2.elapsed_time(e2)
-    if pg:
-        t = torch.tensor([ms2], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms2 = t.item()
+    ms2 = max_over_ranks([s2.elapsed_time(e2)], device=dev)[0]
     h2d = sum(2 * K for (_, _, K, _, _) in first)
     d2h = sum(2 * N for (_, _, _, N, _) in first)
 
@@ -280,11 +274,18 @@ def run_ours(args):
     }
     out["clocks"] = clk.summary()
     if not args.no_prefill:
-        out["prefill"] = {"workload": "config-4 block of 7 projections (q,k,v,o,gate,up,down), W4A16 dequant GEMM on "
-                                      "tcgen05 (kernel gemm_tcgen05_kernel), bf16 X ~N(0,1)",
-                          "peak_bf16_tflops": {"burst": peaks["bf16"], "sustained": peaks["bf16_sustained"],
-                                               "source": peaks["source"]},
+        out["prefill"] = {"workload": "block of 7 projections (q,k,v,o,gate,up,down) at M rows: INT4 g64 and NVFP4 "
+                                      "W4A16 (gemm_tcgen05_kernel, bf16 tcgen05), NVFP4 W4A4 (activation pack + "
+                                      "gemm_fp4_kernel, block-scaled FP4 tcgen05); bf16 X ~N(0,1)",
+                          "peak_tflops": {"bf16_burst": peaks["bf16"], "bf16_sustained": peaks["bf16_sustained"],
+                                          "fp4_burst": peaks["fp4"], "fp4_sustained": peaks["fp4_sustained"],
+                                          "source": peaks["source"] + " bf16; fp4 = 4 x bf16 (nominal dense ratio)"},
                           "results": prefill_measure(wq, synth, torch, dev, peaks, rank=rank)}
+    if not args.no_aux:
+        out["quantize"] = {"workload": "7 projections of one block: INT4 g64 with AWQ scale, NVFP4",
+                           "results": quant_measure(wq, synth, torch, dev, peaks)}
+        out["awq_search"] = {"workload": "7 projections, 512 Student-t calibration tokens, 20 alphas, G=64",
+                             "results": awq_measure(wq, synth, torch, dev, peaks)}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
     if pg:
@@ -300,24 +301,30 @@ def prefill_measure(wq, synth, torch, dev, peaks, Ms=(512, 2048, 8192), reps=20,
     (rotating 2 weight copies) and timed with CUDA events.  Returns TFLOP/s
     per (format, M) over the whole block and per projection."""
     out = {}
-    for fmt in ("int4_g64", "nvfp4"):
+    for fmt in ("int4_g64", "nvfp4", "nvfp4_w4a4"):
         packs = []
         for copy in range(2):
             row = []
             for name, K, N in synth.PROJECTIONS:
                 W = synth.weight(N, K, seed=synth.layer_seed(4, 10 * copy + K + N + 1000 * rank), device=dev)
-                row.append((name, K, N, wq.wq_quantize_nvfp4(W) if fmt == "nvfp4" else wq.wq_quantize_int4(W, 64, 1)))
+                row.append((name, K, N, wq.wq_quantize_int4(W, 64, 1) if fmt == "int4_g64" else wq.wq_quantize_nvfp4(W)))
                 del W
             packs.append(row)
         for M in Ms:
             Xs = {K: synth.activations(M, K, seed=synth.layer_seed(4, M + K), device=dev) for _, K, _ in synth.PROJECTIONS}
             Ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _, _, N in synth.PROJECTIONS}
+            ws = None
+            if fmt == "nvfp4_w4a4":
+                need = max(wq.linear_workspace_size(M, N, K, wq.WQ_FMT_NVFP4, 1) for _, K, N in synth.PROJECTIONS)
+                ws = torch.empty(need, dtype=torch.uint8, device=dev)
             per = {}
             tot_flop, tot_s = 0.0, 0.0
             for j, (name, K, N, _) in enumerate(packs[0]):
                 def call(p, K=K, N=N):
                     if fmt == "nvfp4":
                         wq.wq_linear_nvfp4(Xs[K], p, out=Ys[N])
+                    elif fmt == "nvfp4_w4a4":
+                        wq.wq_linear_nvfp4(Xs[K], p, act_fp4=1, out=Ys[N], ws=ws)
                     else:
                         wq.wq_linear_int4(Xs[K], p, out=Ys[N])
                 call(packs[0][j][3])
@@ -341,13 +348,70 @@ def prefill_measure(wq, synth, torch, dev, peaks, Ms=(512, 2048, 8192), reps=20,
                 tot_s += sec
                 del g
             tf = tot_flop / tot_s / 1e12
-            out[f"{fmt}_M{M}"] = {"TFLOP/s": round(tf, 1), "frac_of_bf16_sustained": round(tf / peaks["bf16_sustained"], 4),
-                                  "frac_of_bf16_burst": round(tf / peaks["bf16"], 4), "per_projection_TFLOP/s": per,
-                                  "us_per_block": round(tot_s * 1e6, 1)}
-            del Xs, Ys
+            pk = peaks["fp4"] if fmt == "nvfp4_w4a4" else peaks["bf16"]
+            pks = peaks["fp4_sustained"] if fmt == "nvfp4_w4a4" else peaks["bf16_sustained"]
+            out[f"{fmt}_M{M}"] = {"TFLOP/s": round(tf, 1), "peak": "fp4" if fmt == "nvfp4_w4a4" else "bf16",
+                                  "frac_of_sustained": round(tf / pks, 4), "frac_of_burst": round(tf / pk, 4),
+                                  "per_projection_TFLOP/s": per, "us_per_block": round(tot_s * 1e6, 1)}
+            del Xs, Ys, ws
         del packs
     torch.cuda.empty_cache()
     return out
+
+
+def quant_measure(wq, synth, torch, dev, peaks, reps=10):
+    """Stage-1 throughput on the 7 projections of one block: INT4 g64 with an
+    AWQ scale, and NVFP4.  GB/s counts bf16 weights read + packed bytes written."""
+    Ws = [synth.weight(N, K, seed=synth.layer_seed(5, i), device=dev) for i, (_, K, N) in enumerate(synth.PROJECTIONS)]
+    Ss = [synth.act_mean_lognormal(W.shape[1], seed=i, device=dev).sqrt() for i, W in enumerate(Ws)]
+    out = {}
+    for fmt in ("int4_g64_awq", "nvfp4"):
+        def run():
+            for W, s_ in zip(Ws, Ss):
+                if fmt == "nvfp4":
+                    wq.wq_quantize_nvfp4(W)
+                else:
+                    wq.wq_quantize_int4(W, 64, 1, s_)
+        run()
+        torch.cuda.synchronize()
+        nbytes = 0
+        for W in Ws:
+            N, K = W.shape
+            nbytes += 2 * N * K + (N * K // 2 + N * K // 16 if fmt == "nvfp4" else sum(wq.int4_sizes(N, K, 64)))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            run()
+        b.record()
+        torch.cuda.synchronize()
+        sec = a.elapsed_time(b) * 1e-3 / reps
+        out[fmt] = {"GB/s": round(nbytes / sec / 1e9, 1), "frac_of_hbm": round(nbytes / sec / 1e9 / peaks["hbm"], 4),
+                    "us_per_block": round(sec * 1e6, 1)}
+    return out
+
+
+def awq_measure(wq, synth, torch, dev, peaks, T=512):
+    """AWQ grid search of the 7 projections (20 alphas, G=64, T calibration tokens)."""
+    alphas = torch.tensor(synth.ALPHA_GRID, dtype=torch.float32, device=dev)
+    tot_s, tot_flop, per = 0.0, 0.0, {}
+    for i, (name, K, N) in enumerate(synth.PROJECTIONS):
+        W = synth.weight(N, K, seed=synth.layer_seed(3, K + N), device=dev)
+        X = synth.activations_student_t(T, K, seed=synth.layer_seed(3, K), device=dev)
+        wq.awq_search_scale(W, alphas, 64, X=X)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        wq.awq_search_scale(W, alphas, 64, X=X)
+        b.record()
+        torch.cuda.synchronize()
+        sec = a.elapsed_time(b) * 1e-3
+        flop = 2.0 * T * N * (2 * K) * len(synth.ALPHA_GRID)  # loss GEMMs over [hi | lo]
+        per[name] = round(sec * 1e3, 3)
+        tot_s += sec
+        tot_flop += flop
+    return {"ms_per_projection": per, "ms_total": round(tot_s * 1e3, 3),
+            "loss_gemm_TFLOP/s": round(tot_flop / tot_s / 1e12, 1),
+            "frac_of_bf16_sustained": round(tot_flop / tot_s / 1e12 / peaks["bf16_sustained"], 4)}
 
 
 # ---------------------------------------------------------------- oracle arm
@@ -437,6 +501,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-aux", action="store_true", help="skip the quantize and AWQ measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -172,28 +172,44 @@ __global__ void __launch_bounds__(Fp4Shape<BN>::THREADS, 1) gemm_fp4_kernel(cons
     const bool is_b = warp >= 8;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     bool ok = true;
-    for (int kb = 0; kb < nkb; ++kb) {
-      const int s = kb % STAGES, r = kb / STAGES;
-      if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) { ok = false; break; }
+    // Scale words of k-block kb for this lane (16 of them), fetched one
+    // k-block ahead so their latency overlaps the previous stage.
+    auto fetch_sf = [&](int kb, uint32_t (&v)[16], int part) {
       if (!is_b) {
-        uint32_t v[16];
+        if (part > 0) return;  // the X scales of a stage fit one 16-column store
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
-          for (int c = 0; c < 4; ++c) v[4 * t + c] = sf_word(a.sfa, m0 + lane + 32 * c, a.M, 4 * kb + t, ksteps, sf_stride);
-        tmem_st16(tmem + lane_base + sfa_col(s), v);
+          for (int c = 0; c < 4; ++c)
+            v[4 * t + c] = kb < nkb ? sf_word(a.sfa, m0 + lane + 32 * c, a.M, 4 * kb + t, ksteps, sf_stride) : 0u;
       } else {
 #pragma unroll
-        for (int h = 0; h < S::SFB_COLS / 16; ++h) {  // 16 columns per store
-          uint32_t v[16];
-#pragma unroll
-          for (int t2 = 0; t2 < 16; ++t2) {
-            const int col = 16 * h + t2;            // column within the stage's SFB block
-            const int t = col / (BN / 32), c = col % (BN / 32);
-            v[t2] = sf_word(a.sfb, n0 + lane + 32 * c, a.N, 4 * kb + t, ksteps, sf_stride);
-          }
-          tmem_st16(tmem + lane_base + sfb_col(s) + 16 * h, v);
+        for (int t2 = 0; t2 < 16; ++t2) {
+          const int col = 16 * part + t2;  // column within the stage's SFB block
+          const int t = col / (BN / 32), c = col % (BN / 32);
+          v[t2] = kb < nkb ? sf_word(a.sfb, n0 + lane + 32 * c, a.N, 4 * kb + t, ksteps, sf_stride) : 0u;
         }
+      }
+    };
+    constexpr int PARTS = S::SFB_COLS / 16;  // SFB stores of 16 columns (X scales use one)
+    uint32_t nxt[PARTS][16];
+#pragma unroll
+    for (int h = 0; h < PARTS; ++h) fetch_sf(0, nxt[h], h);
+    for (int kb = 0; kb < nkb; ++kb) {
+      const int s = kb % STAGES, r = kb / STAGES;
+      uint32_t cur[PARTS][16];
+#pragma unroll
+      for (int h = 0; h < PARTS; ++h)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) cur[h][i] = nxt[h][i];
+#pragma unroll
+      for (int h = 0; h < PARTS; ++h) fetch_sf(kb + 1, nxt[h], h);
+      if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) { ok = false; break; }
+      if (!is_b) {
+        tmem_st16(tmem + lane_base + sfa_col(s), cur[0]);
+      } else {
+#pragma unroll
+        for (int h = 0; h < PARTS; ++h) tmem_st16(tmem + lane_base + sfb_col(s) + 16 * h, cur[h]);
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();

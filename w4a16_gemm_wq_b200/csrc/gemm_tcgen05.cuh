@@ -303,25 +303,42 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
     const int ng = a.K >> a.log2g;
     const uint32_t zw_stride = (ng + 7) >> 3;
     bool ok = true;
+    // Per-row metadata of k-block kb, fetched one k-block ahead so its global
+    // (L2) latency overlaps the previous k-block's dequantization.
+    auto fetch_meta = [&](int kb, uint32_t& raw_a, uint32_t& raw_b) {
+      raw_a = 0;
+      raw_b = 0x88888888u;
+      if (kb >= nkb) return;
+      if (FMT == GEMM_INT4) {
+        const int g = (kb * kGemmBK) >> a.log2g;
+        raw_a = __ldg(a.scales + int64_t(n) * ng + g);
+        if (a.zeros) raw_b = __ldg(a.zeros + int64_t(n) * zw_stride + (g >> 3));
+      } else if (FMT == GEMM_NVFP4) {
+        const int nb = a.K >> 4;
+        const uint8_t* bs = a.bscale + int64_t(n) * nb + kb * 4;
+        const int rem = nb - kb * 4;  // K % 64 == 32 leaves two blocks in the last k-block
+        raw_a = 0;
+        for (int q = 0; q < 4 && q < rem; ++q) raw_a |= uint32_t(__ldg(bs + q)) << (8 * q);
+      }
+    };
+    uint32_t meta_a, meta_b;
+    fetch_meta(0, meta_a, meta_b);
     for (int kb = 0; kb < (FMT == GEMM_BF16_SQ ? 0 : nkb); ++kb) {
       const int s = kb % STAGES, r = kb / STAGES;
-      // metadata first (independent of the stage)
+      const uint32_t cur_a = meta_a, cur_b = meta_b;
+      fetch_meta(kb + 1, meta_a, meta_b);
       uint32_t sc2 = 0, zoff2 = 0;
       float sbv[4] = {0.f, 0.f, 0.f, 0.f};
       if (FMT == GEMM_INT4) {
         const int g = (kb * kGemmBK) >> a.log2g;
-        const float sc = __half2float(__ushort_as_half(__ldg(a.scales + int64_t(n) * ng + g)));
-        int z = 8;
-        if (a.zeros) z = (__ldg(a.zeros + int64_t(n) * zw_stride + (g >> 3)) >> (4 * (g & 7))) & 0xF;
+        const float sc = __half2float(__ushort_as_half(uint16_t(cur_a)));
+        const int z = (cur_b >> (4 * (g & 7))) & 0xF;
         sc2 = pack_bf16x2(sc, sc);
         const uint32_t zb = 0x4300u | uint32_t(z);  // bf16(128 + z)
         zoff2 = zb | (zb << 16);
       } else {
-        const int nb = a.K >> 4;
-        const uint8_t* bs = a.bscale + int64_t(n) * nb + kb * 4;
-        const int rem = nb - kb * 4;  // K % 64 == 32 leaves two blocks in the last k-block
 #pragma unroll
-        for (int q = 0; q < 4; ++q) sbv[q] = q < rem ? e4m3_decode_pos(__ldg(bs + q) & 0x7F) : 0.f;
+        for (int q = 0; q < 4; ++q) sbv[q] = e4m3_decode_pos((cur_a >> (8 * q)) & 0x7F);
       }
       if (!mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag)) { ok = false; break; }
       const uint32_t prow = smem_u32(p_ptr(s)) + uint32_t(t * 32);
