@@ -83,7 +83,7 @@ int wq_nvfp4_sizes(int64_t N, int64_t K, size_t* codes_bytes, size_t* bscale_byt
 
 /* Scratch bytes wq_linear_int4 / wq_linear_nvfp4 need for an [M, K] x [N, K]
  * problem (format WQ_FMT_*, act_fp4 as in wq_linear_nvfp4).  0 means the call
- * needs no workspace and accepts ws = NULL. */
+ * needs no workspace and accepts ws = NULL (every W4A16 call; W4A4 needs one). */
 int wq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int format, int act_fp4,
                              size_t* bytes);
 
@@ -159,7 +159,9 @@ int awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X,
  *   Y        bf16 [M, N]
  *   ws, ws_bytes: scratch of at least wq_linear_workspace_size bytes (may be
  *            NULL when that size is 0)
- * M <= 16 runs the split-K decode GEMV; larger M runs the tensor-core GEMM. */
+ * M <= 16 runs the split-K CUDA-core decode GEMV (one launch, lowest
+ * latency for a single projection); larger M runs the tensor-core GEMM.
+ * wq_linear_group runs decode projections on the tensor-core decode GEMV. */
 int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* qweight,
                    const uint16_t* scales, const uint32_t* zeros, int group_size, int zero_point,
                    const float* act_inv_s, uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
@@ -174,6 +176,38 @@ int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uin
 int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
                     const uint8_t* bscale, const float* global_scale, int act_fp4,
                     const float* act_inv_s, uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
+
+/* One quantized Linear of a group (W4A16; see wq_linear_int4 / wq_linear_nvfp4
+ * for the meaning of each field).  `format` is WQ_FMT_INT4 or WQ_FMT_NVFP4;
+ * fields of the other format are ignored. */
+typedef struct {
+  int format;
+  int64_t N, K;
+  const uint16_t* X;          /* bf16 [M, K] */
+  const float* act_inv_s;     /* fp32 [K] or NULL */
+  const void* packed;         /* INT4 qweight (uint32 [N, K/8]) or NVFP4 codes (uint8 [N, K/2]) */
+  const uint16_t* scales;     /* INT4 fp16 [N, K/G] */
+  const uint32_t* zeros;      /* INT4 packed zero points, NULL for a symmetric pack */
+  int group_size;             /* INT4: 64 or 128 */
+  int zero_point;             /* INT4: 1 asymmetric, 0 symmetric */
+  const uint8_t* bscale;      /* NVFP4 E4M3 [N, K/16] */
+  const float* global_scale;  /* NVFP4 fp32 [1] */
+  uint16_t* Y;                /* bf16 [M, N] */
+} wq_linear_item;
+
+/* wq_linear_group -- the decode-time (M <= 16) quantized Linears of a group
+ * of independent projections at once, e.g. the projections of one
+ * transformer block that read the same normalised activations ("quantization
+ * primer" section 13: decode is memory-bound, so the weights must stream at
+ * HBM speed; one launch pays the launch and ramp cost once for the whole
+ * group).  Each item's Y is what its single entry point computes.  At M <= 2
+ * the items the tensor-core decode GEMV serves (K % 128 == 0, 16-byte aligned
+ * X / packed / act_inv_s, 4-byte aligned scale data) run as one launch per
+ * kernel variant (INT4 group 64, INT4 group 128, NVFP4), up to 24 items and 8
+ * distinct activation vectors each; the other items run one by one after
+ * them.  Items must not alias each other's outputs.  Needs no workspace.
+ * Returns the first failing item's status. */
+int wq_linear_group(const wq_linear_item* items, int count, int64_t M, void* stream);
 
 /* wq_linear_nvfp4_w4a4_noalloc -- the W4A4 product of wq_linear_nvfp4
  * (act_fp4 = 1) for callers that cannot allocate device memory when they

@@ -41,6 +41,7 @@ SIGNATURES = {
     "wq_linear_int4": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "wq_linear_nvfp4": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "wq_linear_nvfp4_w4a4_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P]),
+    "wq_linear_group": (_I, [_P, _I, _I64, _P]),
     "wq_device_error": (_I, [_P]),
 }
 
@@ -267,6 +268,51 @@ def wq_linear_nvfp4_w4a4_noalloc(X: torch.Tensor, p: PackedNVFP4, act_inv_s=None
                                                _ptr(p.global_scale), _ptr(s), _ptr(Y), _stream()),
            "wq_linear_nvfp4_w4a4_noalloc")
     return Y
+
+
+class LinearItem(ctypes.Structure):
+    """Mirror of wq_linear_item (include/wq.h)."""
+
+    _fields_ = [("format", ctypes.c_int), ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("X", ctypes.c_void_p),
+                ("act_inv_s", ctypes.c_void_p), ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("zeros", ctypes.c_void_p), ("group_size", ctypes.c_int), ("zero_point", ctypes.c_int),
+                ("bscale", ctypes.c_void_p), ("global_scale", ctypes.c_void_p), ("Y", ctypes.c_void_p)]
+
+
+def make_group(calls):
+    """(ctypes array of wq_linear_item, M) for [(X, pack, out[, act_inv_s]), ...].
+    Keeps no tensor alive: the caller holds the tensors for as long as the array is used."""
+    arr = (LinearItem * len(calls))()
+    M = None
+    for i, c in enumerate(calls):
+        X, p, Y = c[0], c[1], c[2]
+        inv_s = c[3] if len(c) > 3 else None
+        _dev(X, "X", torch.bfloat16)
+        if M is None:
+            M = X.shape[0]
+        if X.shape != (M, p.K):
+            raise ValueError(f"item {i}: X must be [{M}, {p.K}]")
+        _dev(Y, "out", torch.bfloat16, (M, p.N))
+        s = _opt_f32(inv_s, "act_inv_s", p.K)
+        it = arr[i]
+        it.N, it.K, it.X, it.Y = p.N, p.K, X.data_ptr(), Y.data_ptr()
+        it.act_inv_s = None if s is None else s.data_ptr()
+        if isinstance(p, PackedInt4):
+            it.format, it.packed, it.scales = WQ_FMT_INT4, p.qweight.data_ptr(), p.scales.data_ptr()
+            it.zeros = None if p.zeros is None else p.zeros.data_ptr()
+            it.group_size, it.zero_point = p.group_size, p.zero_point
+        else:
+            it.format, it.packed = WQ_FMT_NVFP4, p.codes.data_ptr()
+            it.bscale, it.global_scale = p.bscale.data_ptr(), p.global_scale.data_ptr()
+    return arr, M
+
+
+def wq_linear_group(calls, group=None):
+    """Run the W4A16 decode Linears [(X, pack, out[, act_inv_s]), ...] of independent
+    projections as one group (one tensor-core GEMV launch per kernel variant for the
+    items it serves)."""
+    arr, M = group if group is not None else make_group(calls)
+    _check(load().wq_linear_group(ctypes.cast(arr, ctypes.c_void_p), len(arr), M, _stream()), "wq_linear_group")
 
 
 def wq_device_error() -> int:

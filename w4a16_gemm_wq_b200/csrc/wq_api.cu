@@ -9,12 +9,14 @@
 
 #include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "wq.h"
 #include "awq.cuh"
 #include "gemm_fp4.cuh"
 #include "gemm_tcgen05.cuh"
 #include "gemv.cuh"
+#include "gemv_tc.cuh"
 #include "quant.cuh"
 #include "wq_common.cuh"
 
@@ -292,6 +294,178 @@ int nvfp4_quantize_launch(const uint16_t* A, int64_t R, int64_t C, const float* 
   return launched("nvfp4_finalize launch");
 }
 
+// ---------------------------------------------------------------- tensor-core decode GEMV
+// One entry of a gemv_tc launch (the single-item calls and wq_linear_group
+// both build these).
+struct TcCall {
+  int fmt;  // wq::FMT_INT4 / wq::FMT_NVFP4
+  int64_t N, K;
+  const uint16_t* X;
+  const float* inv_s;
+  const void* packed;
+  const uint16_t* scales;
+  const uint32_t* zeros;
+  int group_size;
+  const uint8_t* bscale;
+  const float* gscale;
+  uint16_t* Y;
+};
+
+// Kernel variant of a call (-1: gemv_tc does not serve it).  Needs M <= 2,
+// K a multiple of 128 (whole steps), 16-byte aligned codes / X / 1/s and
+// 4-byte aligned scale data.
+int tc_kind(const TcCall& c, int64_t M) {
+  if (M < 1 || M > 2 || c.K % wq::kTcStepK != 0 || c.K > (int64_t(1) << 20)) return -1;
+  if (!aligned16(c.packed) || !aligned16(c.X) || (c.inv_s && !aligned16(c.inv_s))) return -1;
+  const auto a4 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 3) == 0; };
+  if (c.fmt == wq::FMT_INT4) {
+    if (!a4(c.scales) || (c.zeros && !a4(c.zeros))) return -1;
+    return c.group_size == 64 ? wq::TC_INT4_G64 : wq::TC_INT4_G128;
+  }
+  if (!a4(c.bscale)) return -1;
+  return M == 1 ? wq::TC_NVFP4_COLS : wq::TC_NVFP4_MUL;
+}
+
+// Builds one launch over calls of one kind: items with their row-block
+// offsets, distinct activation vectors, the CTAs' row-block ranges (balanced
+// by bytes) and the staged activation bytes the busiest CTA needs.  Returns
+// false when the calls do not fit one launch.
+bool build_tc_args(const TcCall* calls, int count, int64_t M, wq::TcArgs* g, int* nctas, size_t* smem) {
+  if (count < 1 || count > wq::kTcMaxItems) return false;
+  memset(g, 0, sizeof(*g));
+  g->n_items = count;
+  int rb = 0;
+  std::vector<double> cost;
+  for (int i = 0; i < count; ++i) {
+    const TcCall& c = calls[i];
+    wq::TcItem& d = g->items[i];
+    d.packed = static_cast<const uint8_t*>(c.packed);
+    d.scales = c.scales;
+    d.zeros = c.zeros;
+    d.bscale = c.bscale;
+    d.gscale = c.gscale;
+    d.Y = c.Y;
+    d.N = int(c.N);
+    d.K = int(c.K);
+    d.nrb = int((c.N + wq::kTcRows - 1) / wq::kTcRows);
+    d.steps = int(c.K / wq::kTcStepK);
+    d.rb0 = rb;
+    const int xg = c.fmt == wq::FMT_INT4 ? c.group_size : 0;
+    int slot = -1;
+    for (int v = 0; v < g->n_x; ++v)
+      if (g->xs[v].X == c.X && g->xs[v].K == d.K && g->xs[v].inv_s == c.inv_s && g->xs[v].g == xg) slot = v;
+    if (slot < 0) {
+      if (g->n_x == wq::kTcMaxX) return false;
+      slot = g->n_x++;
+      g->xs[slot] = wq::TcX{c.X, c.inv_s, d.K, xg};
+    }
+    d.xslot = slot;
+    // bytes a row block streams (codes + scale data) plus a fixed allowance for its end
+    const double per = wq::kTcRows * (double(c.K / 2) + double(c.K / 64) * 2.5) + 1024.0;
+    for (int r = 0; r < d.nrb; ++r) cost.push_back(per);
+    rb += d.nrb;
+    if (rb >= (1 << 28)) return false;
+  }
+  const int B = std::min(wq::kTcMaxCtas, rb);
+  double total = 0;
+  for (double c : cost) total += c;
+  int b = 0;
+  double accum = 0;
+  g->bounds[0] = 0;
+  for (int r = 0; r < rb; ++r) {
+    accum += cost[size_t(r)];
+    const int left = rb - 1 - r, ctas_left = B - 1 - b;
+    if (b < B - 1 && (accum >= total * (b + 1) / B || left == ctas_left)) g->bounds[++b] = r + 1;
+  }
+  while (b < B - 1) g->bounds[++b] = rb;
+  g->bounds[B] = rb;
+  // staged activations of the busiest CTA
+  const auto item_of = [&](int r) {
+    int i = 0;
+    while (i + 1 < count && g->items[i + 1].rb0 <= r) ++i;
+    return i;
+  };
+  size_t xmax = 0;
+  for (int cb = 0; cb < B; ++cb) {
+    uint32_t used = 0;
+    for (int i = item_of(g->bounds[cb]); i <= item_of(g->bounds[cb + 1] - 1); ++i) used |= 1u << g->items[i].xslot;
+    size_t x = 0;
+    for (int v = 0; v < g->n_x; ++v)
+      if ((used >> v) & 1) x += size_t(wq::tc_x_bytes(g->xs[v].K, g->xs[v].g, int(M)));
+    xmax = std::max(xmax, x);
+  }
+  *smem = xmax;
+  if (*smem > size_t(wq::kTcMaxSmem)) return false;
+  *nctas = B;
+  return true;
+}
+
+template <int M, int KIND>
+int launch_tc_k(const wq::TcArgs& g, int nctas, size_t smem, cudaStream_t st) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemv_tc_kernel<M, KIND>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, wq::kTcMaxSmem),
+                           "gemv_tc smem attribute"))
+      return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nctas, 1, 1);
+  cfg.blockDim = dim3(wq::kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemv_tc_kernel<M, KIND>, g), "gemv_tc launch");
+}
+
+int launch_tc(const wq::TcArgs& g, int64_t M, int kind, int nctas, size_t smem, cudaStream_t st) {
+  if (M == 1) {
+    switch (kind) {
+      case wq::TC_INT4_G64: return launch_tc_k<1, wq::TC_INT4_G64>(g, nctas, smem, st);
+      case wq::TC_INT4_G128: return launch_tc_k<1, wq::TC_INT4_G128>(g, nctas, smem, st);
+      default: return launch_tc_k<1, wq::TC_NVFP4_COLS>(g, nctas, smem, st);
+    }
+  }
+  switch (kind) {
+    case wq::TC_INT4_G64: return launch_tc_k<2, wq::TC_INT4_G64>(g, nctas, smem, st);
+    case wq::TC_INT4_G128: return launch_tc_k<2, wq::TC_INT4_G128>(g, nctas, smem, st);
+    default: return launch_tc_k<2, wq::TC_NVFP4_MUL>(g, nctas, smem, st);
+  }
+}
+
+// Runs calls (each with its kind, -1 = not served) through the tensor-core
+// decode GEMV, one launch per kind (<= kTcMaxItems calls each); done[i]
+// tells which calls it took.
+int run_tc(const TcCall* calls, const int* kinds, int count, int64_t M, cudaStream_t st, char* done) {
+  static thread_local wq::TcArgs g;  // ~3 KB: keep it off the stack
+  for (int i = 0; i < count; ++i) done[i] = 0;
+  for (int kind = 0; kind < 4; ++kind) {
+    for (int start = 0; start < count;) {
+      TcCall sub[wq::kTcMaxItems];
+      int idx[wq::kTcMaxItems];
+      int n = 0, i = start;
+      for (; i < count && n < wq::kTcMaxItems; ++i)
+        if (kinds[i] == kind) {
+          idx[n] = i;
+          sub[n++] = calls[i];
+        }
+      start = i;
+      if (n == 0) break;
+      int nctas = 0;
+      size_t smem = 0;
+      if (!build_tc_args(sub, n, M, &g, &nctas, &smem)) continue;
+      if (int e = launch_tc(g, M, kind, nctas, smem, st)) return e;
+      for (int j = 0; j < n; ++j) done[idx[j]] = 1;
+    }
+  }
+  return WQ_OK;
+}
+
 // Decode GEMV up to this many activation rows, tensor-core GEMM above.
 constexpr int64_t kGemvMaxM = 16;
 
@@ -366,7 +540,11 @@ int wq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int format, int ac
   REQUIRE(format == WQ_FMT_INT4 || format == WQ_FMT_NVFP4, "unknown format %d", format);
   REQUIRE(act_fp4 == 0 || act_fp4 == 1, "act_fp4 must be 0 or 1");
   REQUIRE(!act_fp4 || format == WQ_FMT_NVFP4, "act_fp4 needs the NVFP4 format");
-  *bytes = act_fp4 ? w4a4_layout(M, K).total : 0;
+  if (act_fp4) {
+    *bytes = w4a4_layout(M, K).total;
+  } else {
+    *bytes = 0;
+  }
   return WQ_OK;
 }
 
@@ -519,8 +697,6 @@ int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uin
 int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
                     const uint8_t* bscale, const float* global_scale, int act_fp4, const float* act_inv_s,
                     uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   REQUIRE(M > 0 && M <= (int64_t(1) << 30), "M must be positive");
   if (int e = check_shape(N, K)) return e;
   REQUIRE(act_fp4 == 0 || act_fp4 == 1, "act_fp4 must be 0 or 1");
@@ -556,6 +732,69 @@ int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const ui
   a.X = X; a.inv_s = act_inv_s; a.wq = codes; a.bscale = bscale; a.gscale = global_scale;
   a.Y = Y; a.M = int(M); a.N = int(N); a.K = int(K);
   return launch_gemv<wq::FMT_NVFP4>(a, as_stream(stream));
+}
+
+namespace {
+TcCall tc_call_of(const wq_linear_item& it) {
+  const bool int4 = it.format == WQ_FMT_INT4;
+  return TcCall{int4 ? wq::FMT_INT4 : wq::FMT_NVFP4, it.N, it.K, it.X, it.act_inv_s, it.packed,
+                int4 ? it.scales : nullptr, int4 && it.zero_point ? it.zeros : nullptr, int4 ? it.group_size : 0,
+                int4 ? nullptr : it.bscale, int4 ? nullptr : it.global_scale, it.Y};
+}
+
+int check_items(const wq_linear_item* items, int count, int64_t M) {
+  REQUIRE(items, "items must not be NULL");
+  REQUIRE(count > 0, "count must be positive");
+  REQUIRE(M > 0 && M <= 16, "wq_linear_group serves decode sizes: 1 <= M <= 16 (got %lld)", (long long)M);
+  for (int i = 0; i < count; ++i) {
+    const wq_linear_item& it = items[i];
+    REQUIRE(it.format == WQ_FMT_INT4 || it.format == WQ_FMT_NVFP4, "item %d: unknown format %d", i, it.format);
+    if (int e = check_shape(it.N, it.K)) return e;
+    REQUIRE_PTR(it.X);
+    REQUIRE_PTR(it.packed);
+    REQUIRE_PTR(it.Y);
+    REQUIRE_OPT_PTR(it.act_inv_s);
+    if (it.format == WQ_FMT_INT4) {
+      if (int e = check_group(it.group_size, it.K)) return e;
+      REQUIRE(it.zero_point == 0 || it.zero_point == 1, "item %d: zero_point must be 0 or 1", i);
+      REQUIRE_PTR(it.scales);
+      if (it.zero_point) REQUIRE_PTR(it.zeros);
+    } else {
+      REQUIRE_PTR(it.bscale);
+      REQUIRE_PTR(it.global_scale);
+    }
+  }
+  return WQ_OK;
+}
+}  // namespace
+
+int wq_linear_group(const wq_linear_item* items, int count, int64_t M, void* stream) {
+  if (int e = check_items(items, count, M)) return e;
+  cudaStream_t st = as_stream(stream);
+  // items the tensor-core decode GEMV serves run first (one launch per kernel
+  // variant); the rest, and any that do not fit a launch, one by one
+  std::vector<char> done(static_cast<size_t>(count), 0);
+  if (M <= 2) {
+    std::vector<TcCall> calls(static_cast<size_t>(count));
+    std::vector<int> kinds(static_cast<size_t>(count));
+    for (int i = 0; i < count; ++i) {
+      calls[size_t(i)] = tc_call_of(items[i]);
+      kinds[size_t(i)] = tc_kind(calls[size_t(i)], M);
+    }
+    if (int e = run_tc(calls.data(), kinds.data(), count, M, st, done.data())) return e;
+  }
+  for (int i = 0; i < count; ++i) {
+    if (done[size_t(i)]) continue;
+    const wq_linear_item& it = items[i];
+    const int e = it.format == WQ_FMT_INT4
+                      ? wq_linear_int4(it.X, M, it.N, it.K, static_cast<const uint32_t*>(it.packed), it.scales,
+                                       it.zero_point ? it.zeros : nullptr, it.group_size, it.zero_point, it.act_inv_s,
+                                       it.Y, nullptr, 0, stream)
+                      : wq_linear_nvfp4(it.X, M, it.N, it.K, static_cast<const uint8_t*>(it.packed), it.bscale,
+                                        it.global_scale, 0, it.act_inv_s, it.Y, nullptr, 0, stream);
+    if (e) return e;
+  }
+  return WQ_OK;
 }
 
 int wq_linear_nvfp4_w4a4_noalloc(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
