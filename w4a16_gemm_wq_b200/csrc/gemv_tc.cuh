@@ -10,7 +10,7 @@
 // Step: 16 weight rows ("row block") x 128 k.  Lane (g, c) (g = lane / 4,
 // c = lane % 4) loads 16 bytes (32 codes) of rows g and g + 8 at
 // k = 128 j + 32 c, so every row is read in 64-byte runs and a warp keeps
-// kTcDepth steps (8 KB) in flight in registers.
+// kTcDepth steps (3 KB) in flight in registers.
 //
 // Partition: CTA b owns the row blocks [bounds[b], bounds[b+1]) of the
 // launch (items in order, balanced by bytes on the host); its 8 warps split
@@ -56,9 +56,9 @@ constexpr int kTcMaxItems = 24;
 constexpr int kTcMaxX = 8;        // distinct staged activation vectors
 constexpr int kTcRows = 16;       // rows per row block
 constexpr int kTcStepK = 128;     // k per step
-constexpr int kTcWarps = 8;
+constexpr int kTcWarps = 16;
 constexpr int kTcThreads = kTcWarps * 32;
-constexpr int kTcDepth = 8;       // steps in flight per warp (8 KB)
+constexpr int kTcDepth = 3;       // steps in flight per warp (3 KB; 48 KB per SM)
 constexpr int kTcMaxCtas = 148;
 constexpr int kTcMaxSmem = 200 * 1024;
 
