@@ -90,3 +90,25 @@ def test_m8192_gate_sampled(lib):
     ref = oracle.linear(X[rows].cpu(), _deq(p))
     assert_linear_close(Y[rows], ref, what="int4 gate M=8192")
     assert lib.wq_device_error() == 0
+
+
+@pytest.mark.parametrize("M,N", [(2300, 4200), (2300, 4100), (2300, 2100)])
+@pytest.mark.parametrize("fmt", ["int4_g64", "int4_g128", "int4_sym", "nvfp4"])
+def test_two_accumulator_tiles_ragged(lib, M, N, fmt):
+    # enough tiles for 256-row CTAs (two tensor-memory accumulators sharing each
+    # dequantized W tile): W tiles of 256 (4200, 4100: vector and scalar stores)
+    # and of 128 (2100); M = 2300 leaves a ragged last row band
+    K = 1024
+    W = synth.weight(N, K, seed=M + N, device="cuda")
+    X = synth.activations(M, K, seed=N, device="cuda")
+    inv_s = (1.0 / synth.act_mean_lognormal(K, seed=5).sqrt()).cuda() if fmt == "int4_g128" else None
+    if fmt == "nvfp4":
+        p = lib.wq_quantize_nvfp4(W)
+        Y = lib.wq_linear_nvfp4(X, p)
+    else:
+        p = lib.wq_quantize_int4(W, 128 if fmt == "int4_g128" else 64, 0 if fmt == "int4_sym" else 1)
+        Y = lib.wq_linear_int4(X, p, act_inv_s=inv_s)
+    # the second accumulator of the first tile, a full band around 2048 and the tail
+    rows = np.array(sorted(set(range(120, 264, 3)) | set(range(2040, 2300, 7)) | {M - 1}))
+    ref = oracle.linear(X[rows].cpu(), _deq(p), None if inv_s is None else inv_s.cpu().numpy())
+    assert_linear_close(Y[rows], ref, what=f"{fmt} M={M} N={N}")

@@ -37,10 +37,14 @@ namespace wq {
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 64;
 
-template <int BN>
+// BMT = 128: one M = 128 MMA per k step; BMT = 256: two (rows 0-127 and
+// 128-255 of the X tile) sharing the dequantized W tile, into two tensor-
+// memory accumulators side by side (columns [0, BN) and [BN, 2 BN)), which
+// halves the dequantization per flop.
+template <int BN, int BMT = kGemmBM>
 struct GemmShape {
   static constexpr int STAGES = (BN == 256) ? 3 : 4;
-  static constexpr int A_BYTES = kGemmBM * kGemmBK * 2;  // 16 KB, bf16 X tile
+  static constexpr int A_BYTES = BMT * kGemmBK * 2;      // bf16 X tile (16 or 32 KB)
   static constexpr int B_BYTES = BN * kGemmBK * 2;       // dequantized W tile
   static constexpr int P_BYTES = BN * kGemmBK / 2;       // packed 4-bit W tile
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
@@ -48,6 +52,10 @@ struct GemmShape {
   static constexpr int THREADS = 128 + DEQ_THREADS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr int NACC = BMT / kGemmBM;             // accumulators
+  static constexpr int TMEM_COLS = BN * NACC;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
+  static_assert(TMEM_COLS <= 512, "tensor memory columns");
 };
 
 struct GemmArgs {
@@ -177,17 +185,18 @@ __device__ __forceinline__ uint4 dequant_word_int4(uint32_t w, uint32_t zoff2, u
 }
 
 // NVFP4: one packed word (codes of k = 8j..8j+7, low nibble = even k) -> 8 bf16
-// e2m1 * sb (exact in bf16), natural order.
-__device__ __forceinline__ uint32_t e2m1x2_to_bf16x2_scaled(uint32_t byte, float sb) {
+// e2m1 * sb, natural order.  The product is formed in f16 (exact: at most 6
+// significant bits, |v| <= 6 * 448) and then rounded to bf16 (exact as well).
+__device__ __forceinline__ uint32_t e2m1x2_scaled_bf16x2(uint32_t byte, uint32_t sb2) {
   uint32_t h;
   asm("{ .reg .b8 q; cvt.u8.u32 q, %1; cvt.rn.f16x2.e2m1x2 %0, q; }" : "=r"(h) : "r"(byte));
-  const __half2 hh = *reinterpret_cast<const __half2*>(&h);
-  const float2 f = __half22float2(hh);
-  return pack_bf16x2(f.x * sb, f.y * sb);
+  asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(h) : "r"(sb2));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_bf16x2(f.x, f.y);
 }
-__device__ __forceinline__ uint4 dequant_word_nvfp4(uint32_t w, float sb) {
-  return make_uint4(e2m1x2_to_bf16x2_scaled(w & 0xFF, sb), e2m1x2_to_bf16x2_scaled((w >> 8) & 0xFF, sb),
-                    e2m1x2_to_bf16x2_scaled((w >> 16) & 0xFF, sb), e2m1x2_to_bf16x2_scaled(w >> 24, sb));
+__device__ __forceinline__ uint4 dequant_word_nvfp4(uint32_t w, uint32_t sb2) {
+  return make_uint4(e2m1x2_scaled_bf16x2(w & 0xFF, sb2), e2m1x2_scaled_bf16x2((w >> 8) & 0xFF, sb2),
+                    e2m1x2_scaled_bf16x2((w >> 16) & 0xFF, sb2), e2m1x2_scaled_bf16x2(w >> 24, sb2));
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
@@ -200,9 +209,11 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   return v;
 }
 
-template <int FMT, int BN>
-__global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel(const __grid_constant__ GemmArgs a) {
-  using S = GemmShape<BN>;
+template <int FMT, int BN, int BMT = kGemmBM>
+__global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
+    gemm_tcgen05_kernel(const __grid_constant__ GemmArgs a) {
+  using S = GemmShape<BN, BMT>;
+  static_assert(FMT != GEMM_BF16_SQ || BMT == kGemmBM, "the sum-of-squares epilogue uses one accumulator");
   constexpr int STAGES = S::STAGES;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled operand tiles
@@ -222,7 +233,7 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * BN;
+  const int m0 = blockIdx.y * BMT, n0 = blockIdx.x * BN;
   const int nkb = (a.K + kGemmBK - 1) / kGemmBK;
   constexpr int DEQ_WARP0 = 4;
   constexpr int DEQ_WARPS = S::DEQ_THREADS / 32;
@@ -240,7 +251,7 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
     prefetch_tmap(&a.tmP);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -290,8 +301,12 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
         const uint64_t ad = desc_kmajor_sw128(a_addr(s));
         const uint64_t bd = desc_kmajor_sw128(b_addr(s));
 #pragma unroll
-        for (int kk = 0; kk < kGemmBK / 16; ++kk)  // +32 bytes per K=16 step inside the swizzle atom
+        for (int kk = 0; kk < kGemmBK / 16; ++kk) {  // +32 bytes per K=16 step inside the swizzle atom
           umma_bf16(tmem_acc, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), IDESC, (kb | kk) != 0);
+          if (S::NACC == 2)  // rows 128-255 of the X tile start 16 KB (16 atoms) further
+            umma_bf16(tmem_acc + BN, desc_kmajor_sw128(a_addr(s) + 16384) + uint64_t(2 * kk),
+                      bd + uint64_t(2 * kk), IDESC, (kb | kk) != 0);
+        }
         umma_commit(&empty[s]);
       }
       umma_commit(accum);  // also on abort: completes when issued MMAs are done
@@ -328,7 +343,7 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
       const uint32_t cur_a = meta_a, cur_b = meta_b;
       fetch_meta(kb + 1, meta_a, meta_b);
       uint32_t sc2 = 0, zoff2 = 0;
-      float sbv[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t sbv[4] = {0, 0, 0, 0};  // NVFP4: the k-block's 4 E4M3 block scales as f16x2 {sb, sb}
       if (FMT == GEMM_INT4) {
         const int g = (kb * kGemmBK) >> a.log2g;
         const float sc = __half2float(__ushort_as_half(uint16_t(cur_a)));
@@ -338,7 +353,13 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
         zoff2 = zb | (zb << 16);
       } else {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) sbv[q] = e4m3_decode_pos((cur_a >> (8 * q)) & 0x7F);
+        for (int q = 0; q < 4; q += 2) {  // two E4M3 bytes -> f16x2 (exact), then replicate each
+          uint32_t h2;
+          asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }"
+              : "=r"(h2) : "r"((cur_a >> (8 * q)) & 0x7F7Fu));
+          sbv[q] = __byte_perm(h2, 0, 0x1010);
+          sbv[q + 1] = __byte_perm(h2, 0, 0x3232);
+        }
       }
       if (!mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag)) { ok = false; break; }
       const uint32_t prow = smem_u32(p_ptr(s)) + uint32_t(t * 32);
@@ -370,15 +391,18 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
     go = __all_sync(0xffffffffu, go);  // tcgen05.ld below is warp-collective
     if (go) {
       tc_fence_after();
-      const int quarter = warp & 3;                // TMEM lanes 32*quarter .. +31
-      const int col0 = ((warp - DEQ_WARP0) >> 2) * 128;  // two warps per quarter when BN = 256
-      const int row = m0 + quarter * 32 + lane;
+      const int quarter = warp & 3;                      // TMEM lanes 32*quarter .. +31
+      constexpr int WPQ = DEQ_WARPS / 4;                 // epilogue warps per lane quarter
+      const int wi = (warp - DEQ_WARP0) >> 2;            // this warp's index among them
       const float gmul = (FMT == GEMM_NVFP4) ? __ldg(a.gscale) : 1.0f;
       const bool vec = (a.N % 8) == 0;
       double sq = 0.0;
-      for (int c = col0; c < min(col0 + 128, BN); c += 32) {
+      // (accumulator, 32-column chunk) units of this quarter, dealt round-robin
+      for (int u = wi; u < S::NACC * (BN / 32); u += WPQ) {
+        const int acc = u / (BN / 32), c = (u % (BN / 32)) * 32;
+        const int row = m0 + acc * kGemmBM + quarter * 32 + lane;
         uint32_t v[32];
-        tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(c), v);
+        tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN + c), v);
         if (FMT == GEMM_BF16_SQ) {
           float part = 0.f;
           if (row < a.M) {
@@ -426,7 +450,7 @@ __global__ void __launch_bounds__(GemmShape<BN>::THREADS, 1) gemm_tcgen05_kernel
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_acc, BN);
+    tmem_dealloc(tmem_acc, S::TMEM_COLS);
   }
 }
 

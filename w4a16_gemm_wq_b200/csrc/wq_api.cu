@@ -157,19 +157,19 @@ int make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int e
 }
 
 // ---------------------------------------------------------------- GEMM launch
-template <int FMT, int BN>
+template <int FMT, int BN, int BMT = wq::kGemmBM>
 int launch_gemm_prepared(const wq::GemmArgs& a, cudaStream_t st) {
-  using S = wq::GemmShape<BN>;
+  using S = wq::GemmShape<BN, BMT>;
   static bool attr_set = false;  // per instantiation; the value is the same on every device
   if (!attr_set) {
-    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_tcgen05_kernel<FMT, BN>,
+    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_tcgen05_kernel<FMT, BN, BMT>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES),
                            "gemm smem attribute"))
       return e;
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((a.N + BN - 1) / BN, (a.M + wq::kGemmBM - 1) / wq::kGemmBM, 1);
+  cfg.gridDim = dim3((a.N + BN - 1) / BN, (a.M + BMT - 1) / BMT, 1);
   cfg.blockDim = dim3(S::THREADS, 1, 1);
   cfg.dynamicSmemBytes = S::SMEM_BYTES;
   cfg.stream = st;
@@ -178,24 +178,32 @@ int launch_gemm_prepared(const wq::GemmArgs& a, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemm_tcgen05_kernel<FMT, BN>, a), "gemm launch");
+  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemm_tcgen05_kernel<FMT, BN, BMT>, a), "gemm launch");
 }
 
-template <int FMT, int BN>
+template <int FMT, int BN, int BMT = wq::kGemmBM>
 int launch_gemm_bn(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaStream_t st) {
-  if (int e = make_tmap_2d(&a.tmA, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(a.M), uint64_t(a.K),
-                           wq::kGemmBM, wq::kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (int e = make_tmap_2d(&a.tmA, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(a.M), uint64_t(a.K), BMT,
+                           wq::kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B))
     return e;
   if (int e = make_tmap_2d(&a.tmP, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 2), BN,
                            wq::kGemmBK / 2, CU_TENSOR_MAP_SWIZZLE_NONE))
     return e;
-  return launch_gemm_prepared<FMT, BN>(a, st);
+  return launch_gemm_prepared<FMT, BN, BMT>(a, st);
 }
 
 int gemm_bn(int64_t M, int64_t N);
 
+// Tile of the quantized GEMM.  A 256-row CTA (two accumulators sharing each
+// dequantized W tile) does twice the flops of a 128-row one for the same
+// dequantization, so one wave of them is never slower than two waves of
+// 128-row tiles: use it while it still covers about two thirds of the SMs,
+// with the widest W tile that does; else 128 rows.
 template <int FMT>
 int launch_gemm(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaStream_t st) {
+  const auto tiles = [&](int bm, int bn) { return ((a.N + bn - 1) / bn) * int64_t((a.M + bm - 1) / bm); };
+  if (tiles(256, 256) >= 100) return launch_gemm_bn<FMT, 256, 256>(a, X, packed, st);
+  if (tiles(256, 128) >= 100) return launch_gemm_bn<FMT, 128, 256>(a, X, packed, st);
   if (gemm_bn(a.M, a.N) == 256) return launch_gemm_bn<FMT, 256>(a, X, packed, st);
   return launch_gemm_bn<FMT, 128>(a, X, packed, st);
 }
