@@ -11,12 +11,15 @@
 //
 // One CTA = one 128 x BN output tile; k-blocks of 256 elements (128 bytes of
 // packed E2M1 per row = one 128-byte swizzle atom), STAGES deep:
-//   warp 0      TMA: packed X tile [128 x 128 B] and W tile [BN x 128 B]
+//   warp 0      TMA: packed X tile [128 x 128 B] and W tile [BN x 128 B], and
+//               (K % 256 == 0) their E4M3 scale tiles [rows x 16 B]
 //   warp 1      TMEM allocation (512 columns) and the tcgen05.mma issuer
 //               (4 MMAs of K = 64 per k-block)
 //   warps 4..11 copy the stage's E4M3 scales into tensor memory with
-//               tcgen05.st (warps 4-7: X scales, 8-11: W scales), then run the
-//               epilogue (tcgen05.ld, x g_x g_w, bf16 store).
+//               tcgen05.st (warps 4-7: X scales, 8-11: W scales), reading
+//               them from the stage in shared memory (or, when K is not a
+//               multiple of 256, from global memory one k-block ahead), then
+//               run the epilogue (tcgen05.ld, x g_x g_w, bf16 store).
 // Scale-factor placement in tensor memory: the four scales (4 bytes) of row r
 // for one K = 64 step form one 32-bit word at column (r / 32) and lane
 // (r % 32) of every 32-lane subpartition.
@@ -33,7 +36,9 @@ struct Fp4Shape {
   static constexpr int STAGES = 4;
   static constexpr int A_BYTES = kGemmBM * kFp4BK / 2;  // 16 KB
   static constexpr int B_BYTES = BN * kFp4BK / 2;       // 32 KB at BN = 256
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SA_BYTES = kGemmBM * 16;         // X scales of the k-block: 16 B per row
+  static constexpr int SB_BYTES = BN * 16;              // W scales
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SA_BYTES + SB_BYTES;
   static constexpr int THREADS = 384;
   static constexpr int SFA_COLS = 4 * 4;         // 4 K-steps x 4 row blocks of 32
   static constexpr int SFB_COLS = 4 * (BN / 32);
@@ -41,11 +46,16 @@ struct Fp4Shape {
   static constexpr int TMEM_COLS = 512;
   static_assert(256 + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+  static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory of one CTA");
 };
 
 struct Fp4Args {
   CUtensorMap tmA;        // X codes u8 [M, K/2], box {128 B, 128}, 128B swizzle
   CUtensorMap tmB;        // W codes u8 [N, K/2], box {128 B, BN}, 128B swizzle
+  CUtensorMap tmSA;       // X scales u8 [M, K/16], box {16 B, 128} (used iff sf_tma)
+  CUtensorMap tmSB;       // W scales u8 [N, K/16], box {16 B, BN} (used iff sf_tma)
+  int sf_tma;             // scale rows 16-byte aligned (K % 256 == 0): scales arrive with the stage
   const uint8_t* sfa;     // X e4m3 [M, K/16]
   const uint8_t* sfb;     // W e4m3 [N, K/16]
   const float* gx;        // fp32 [1]
@@ -117,6 +127,10 @@ __global__ void __launch_bounds__(Fp4Shape<BN>::THREADS, 1) gemm_fp4_kernel(cons
     fence_mbar_init();
     prefetch_tmap(&a.tmA);
     prefetch_tmap(&a.tmB);
+    if (a.sf_tma) {
+      prefetch_tmap(&a.tmSA);
+      prefetch_tmap(&a.tmSB);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -139,9 +153,14 @@ __global__ void __launch_bounds__(Fp4Shape<BN>::THREADS, 1) gemm_fp4_kernel(cons
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = kb % STAGES, r = kb / STAGES;
         if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) break;
-        mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
-        tma_load_2d(smem + s * S::STAGE_BYTES, &a.tmA, &full[s], kb * (kFp4BK / 2), m0);
-        tma_load_2d(smem + s * S::STAGE_BYTES + S::A_BYTES, &a.tmB, &full[s], kb * (kFp4BK / 2), n0);
+        uint8_t* st = smem + s * S::STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[s], a.sf_tma ? S::STAGE_BYTES : S::A_BYTES + S::B_BYTES);
+        tma_load_2d(st, &a.tmA, &full[s], kb * (kFp4BK / 2), m0);
+        tma_load_2d(st + S::A_BYTES, &a.tmB, &full[s], kb * (kFp4BK / 2), n0);
+        if (a.sf_tma) {  // 16 bytes = the 16 scales of the k-block's 256 elements, per row
+          tma_load_2d(st + S::A_BYTES + S::B_BYTES, &a.tmSA, &full[s], kb * 16, m0);
+          tma_load_2d(st + S::A_BYTES + S::B_BYTES + S::SA_BYTES, &a.tmSB, &full[s], kb * 16, n0);
+        }
         ++issued;
       }
       if (*abort_flag) {
@@ -192,18 +211,52 @@ __global__ void __launch_bounds__(Fp4Shape<BN>::THREADS, 1) gemm_fp4_kernel(cons
       }
     };
     constexpr int PARTS = S::SFB_COLS / 16;  // SFB stores of 16 columns (X scales use one)
-    uint32_t nxt[PARTS][16];
+    // Scale words of k-block kb from the stage in shared memory: row r's 16
+    // bytes are its 4 words (K = 64 steps t); column (rows/32) t + c of lane l
+    // takes row 32 c + l (conflict-free 16-byte reads, consecutive rows per lane).
+    auto stage_sf = [&](int s, uint32_t (&v)[16], int part) {
+      const uint32_t base = sbase + uint32_t(s * S::STAGE_BYTES + S::A_BYTES + S::B_BYTES);
+      if (!is_b) {
+        if (part > 0) return;
 #pragma unroll
-    for (int h = 0; h < PARTS; ++h) fetch_sf(0, nxt[h], h);
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = ld_shared_v4(base + uint32_t((32 * c + lane) * 16));
+          v[c] = w.x; v[4 + c] = w.y; v[8 + c] = w.z; v[12 + c] = w.w;
+        }
+      } else {
+        constexpr int G = BN / 32;  // row groups of 32
+#pragma unroll
+        for (int t2 = 0; t2 < 16; t2 += 4) {
+          // columns 16 part + t2 .. +3 share k-step t when G >= 4: t = col / G, c = col % G
+          const int col = 16 * part + t2, t = col / G, c0 = col % G;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 w = ld_shared_v4(base + uint32_t(S::SA_BYTES + (32 * (c0 + q) + lane) * 16));
+            v[t2 + q] = t == 0 ? w.x : t == 1 ? w.y : t == 2 ? w.z : w.w;
+          }
+        }
+      }
+    };
+    uint32_t nxt[PARTS][16];
+    if (!a.sf_tma) {
+#pragma unroll
+      for (int h = 0; h < PARTS; ++h) fetch_sf(0, nxt[h], h);
+    }
     for (int kb = 0; kb < nkb; ++kb) {
       const int s = kb % STAGES, r = kb / STAGES;
       uint32_t cur[PARTS][16];
+      if (a.sf_tma) {
+        if (!mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag)) { ok = false; break; }
 #pragma unroll
-      for (int h = 0; h < PARTS; ++h)
+        for (int h = 0; h < PARTS; ++h) stage_sf(s, cur[h], h);
+      } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) cur[h][i] = nxt[h][i];
+        for (int h = 0; h < PARTS; ++h)
 #pragma unroll
-      for (int h = 0; h < PARTS; ++h) fetch_sf(kb + 1, nxt[h], h);
+          for (int i = 0; i < 16; ++i) cur[h][i] = nxt[h][i];
+#pragma unroll
+        for (int h = 0; h < PARTS; ++h) fetch_sf(kb + 1, nxt[h], h);
+      }
       if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) { ok = false; break; }
       if (!is_b) {
         tmem_st16(tmem + lane_base + sfa_col(s), cur[0]);

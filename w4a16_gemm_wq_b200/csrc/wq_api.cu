@@ -264,6 +264,16 @@ int launch_fp4_bn(wq::Fp4Args& a, const uint8_t* xcodes, const uint8_t* wcodes, 
   if (int e = make_tmap_2d(&a.tmB, wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 2), BN,
                            wq::kFp4BK / 2, CU_TENSOR_MAP_SWIZZLE_128B))
     return e;
+  // scale tiles ride with the stage when their rows are 16-byte aligned
+  a.sf_tma = (a.K % wq::kFp4BK == 0) && aligned16(a.sfa) && aligned16(a.sfb);
+  if (a.sf_tma) {
+    if (int e = make_tmap_2d(&a.tmSA, a.sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.M), uint64_t(a.K / 16),
+                             wq::kGemmBM, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return e;
+    if (int e = make_tmap_2d(&a.tmSB, a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 16), BN,
+                             16, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return e;
+  }
   static bool attr_set = false;
   if (!attr_set) {
     if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_fp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
