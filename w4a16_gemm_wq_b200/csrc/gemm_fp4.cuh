@@ -20,6 +20,8 @@
 //               them from the stage in shared memory (or, when K is not a
 //               multiple of 256, from global memory one k-block ahead), then
 //               run the epilogue (tcgen05.ld, x g_x g_w, bf16 store).
+// With K a multiple of 256 the host launches the persistent variant below
+// instead.
 // Scale-factor placement in tensor memory: the four scales (4 bytes) of row r
 // for one K = 64 step form one 32-bit word at column (r / 32) and lane
 // (r % 32) of every 32-lane subpartition.
@@ -300,6 +302,230 @@ __global__ void __launch_bounds__(Fp4Shape<BN>::THREADS, 1) gemm_fp4_kernel(cons
           }
         }
       }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, S::TMEM_COLS);
+  }
+}
+
+}  // namespace wq
+
+namespace wq {
+
+// ---------------------------------------------------------------------------
+// Persistent variant (scale tiles by TMA, i.e. K % 256 == 0): one CTA per SM
+// walks the output tiles t = blockIdx.x, + gridDim.x, ... (N fastest, so
+// consecutive tiles of a CTA reuse the X rows in L2).  The TMA / scale /
+// MMA pipeline runs on across tiles, and two 128-column accumulators in
+// tensor memory alternate, so the epilogue warps drain tile i while the
+// MMAs of tile i + 1 proceed:
+//   warp 0      TMA producer (codes and scale tiles, STAGES deep)
+//   warp 1      TMEM allocation and the MMA issuer
+//   warps 4..7  copy each stage's X and W scales into tensor memory (one lane
+//               quarter each; every quarter holds the full 128-row block)
+//   warps 8..11 epilogue of one lane quarter each (tcgen05.ld, x g_x g_w, bf16)
+// Tensor memory: accumulators at columns [0, 256), then STAGES x 32 scale columns.
+constexpr int kFp4PBN = 128;
+
+struct Fp4PShape {
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = kGemmBM * kFp4BK / 2;      // 16 KB
+  static constexpr int B_BYTES = kFp4PBN * kFp4BK / 2;      // 16 KB
+  static constexpr int SA_BYTES = kGemmBM * 16;
+  static constexpr int SB_BYTES = kFp4PBN * 16;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SA_BYTES + SB_BYTES;  // 36 KB
+  static constexpr int THREADS = 384;
+  static constexpr int SFA_COLS = 16;                       // 4 K-steps x 4 row blocks of 32
+  static constexpr int SFB_COLS = 16;                       // 4 K-steps x 4 row blocks of 32
+  static constexpr int SF_STAGE_COLS = SFA_COLS + SFB_COLS;
+  static constexpr int ACC_COLS = 2 * kFp4PBN;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(ACC_COLS + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+  static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
+};
+
+__global__ void __launch_bounds__(Fp4PShape::THREADS, 1) gemm_fp4_persistent_kernel(const __grid_constant__ Fp4Args a) {
+  using S = Fp4PShape;
+  constexpr int STAGES = S::STAGES;
+  constexpr int BN = kFp4PBN;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+  uint64_t* full = bars;                    // TMA landed (codes + scales)
+  uint64_t* sfready = bars + STAGES;        // scales in tensor memory
+  uint64_t* empty = bars + 2 * STAGES;      // MMAs of the stage finished
+  uint64_t* acc_full = bars + 3 * STAGES;   // [2] accumulator complete
+  uint64_t* acc_empty = acc_full + 2;       // [2] accumulator drained by the epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nkb = (a.K + kFp4BK - 1) / kFp4BK;
+  const int n_tiles = (a.N + BN - 1) / BN, m_tiles = (a.M + kGemmBM - 1) / kGemmBM;
+  const int tiles = n_tiles * m_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&sfready[s], 4);  // the 4 scale-copy warps
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);  // the 4 epilogue warps
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&a.tmA);
+    prefetch_tmap(&a.tmB);
+    prefetch_tmap(&a.tmSA);
+    prefetch_tmap(&a.tmSB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto sfa_col = [&](int s) { return uint32_t(S::ACC_COLS + s * S::SF_STAGE_COLS); };
+  auto sfb_col = [&](int s) { return uint32_t(S::ACC_COLS + s * S::SF_STAGE_COLS + S::SFA_COLS); };
+
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      int q = 0;  // global k-block sequence number of this CTA
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int m0 = (t / n_tiles) * kGemmBM, n0 = (t % n_tiles) * BN;
+        for (int kb = 0; kb < nkb; ++kb, ++q) {
+          const int s = q % STAGES, r = q / STAGES;
+          if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) { ok = false; break; }
+          uint8_t* st = smem + s * S::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], S::STAGE_BYTES);
+          tma_load_2d(st, &a.tmA, &full[s], kb * (kFp4BK / 2), m0);
+          tma_load_2d(st + S::A_BYTES, &a.tmB, &full[s], kb * (kFp4BK / 2), n0);
+          tma_load_2d(st + S::A_BYTES + S::B_BYTES, &a.tmSA, &full[s], kb * 16, m0);
+          tma_load_2d(st + S::A_BYTES + S::B_BYTES + S::SA_BYTES, &a.tmSB, &full[s], kb * 16, n0);
+        }
+      }
+      if (!ok) {  // let copies already issued land before the CTA leaves
+        for (int k = (q > STAGES ? q - STAGES : 0); k < q; ++k)
+          mbar_wait(&full[k % STAGES], (k / STAGES) & 1, ERR_TIMEOUT_TMA, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_nvf4(kGemmBM, BN);
+      int q = 0, i = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++i) {
+        const int b = i & 1, u = i >> 1;
+        if (u > 0 && !mbar_wait(&acc_empty[b], (u - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dacc = tmem + uint32_t(b * BN);
+        for (int kb = 0; kb < nkb; ++kb, ++q) {
+          const int s = q % STAGES, r = q / STAGES;
+          if (!mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag) ||
+              !mbar_wait(&sfready[s], r & 1, ERR_TIMEOUT_PIPE, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = desc_kmajor_sw128(sbase + uint32_t(s * S::STAGE_BYTES));
+          const uint64_t bd = desc_kmajor_sw128(sbase + uint32_t(s * S::STAGE_BYTES + S::A_BYTES));
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            umma_nvf4(dacc, ad + uint64_t(2 * k4), bd + uint64_t(2 * k4), IDESC, tmem + sfa_col(s) + 4 * k4,
+                      tmem + sfb_col(s) + 4 * k4, (kb | k4) != 0);
+          umma_commit(&empty[s]);
+        }
+        umma_commit(&acc_full[b]);  // also after an abort: completes when the issued MMAs are done
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------------------- scales -> tensor memory
+    const int quarter = warp & 3;
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    int q = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      for (int kb = 0; kb < nkb; ++kb, ++q) {
+        const int s = q % STAGES, r = q / STAGES;
+        if (!mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag)) { ok = false; break; }
+        // row r of a scale tile: its 4 words (K = 64 steps k4); column 4 k4 + c of
+        // lane l takes row 32 c + l
+        const uint32_t base = sbase + uint32_t(s * S::STAGE_BYTES + S::A_BYTES + S::B_BYTES);
+        uint32_t va[16], vb[16];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 wa = ld_shared_v4(base + uint32_t((32 * c + lane) * 16));
+          const uint4 wb = ld_shared_v4(base + uint32_t(S::SA_BYTES + (32 * c + lane) * 16));
+          va[c] = wa.x; va[4 + c] = wa.y; va[8 + c] = wa.z; va[12 + c] = wa.w;
+          vb[c] = wb.x; vb[4 + c] = wb.y; vb[8 + c] = wb.z; vb[12 + c] = wb.w;
+        }
+        if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) { ok = false; break; }
+        tmem_st16(tmem + lane_base + sfa_col(s), va);
+        tmem_st16(tmem + lane_base + sfb_col(s), vb);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sfready[s]);
+      }
+    }
+  } else if (warp >= 8) {
+    // ---------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    const uint32_t lane_base = uint32_t(quarter * 32) << 16;
+    const float gmul = __ldg(a.gx) * __ldg(a.gw);
+    const bool vec = (a.N % 8) == 0;
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int b = i & 1, u = i >> 1;
+      bool go = mbar_wait(&acc_full[b], u & 1, ERR_TIMEOUT_MMA, abort_flag);
+      go = __all_sync(0xffffffffu, go);  // tcgen05.ld is warp-collective
+      if (!go) break;
+      tc_fence_after();
+      const int m0 = (t / n_tiles) * kGemmBM, n0 = (t % n_tiles) * BN;
+      const int row = m0 + quarter * 32 + lane;
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + uint32_t(b * BN + c), v);
+        if (row < a.M) {
+          uint16_t* yrow = a.Y + int64_t(row) * a.N;
+          const int nb = n0 + c;
+          if (vec && nb + 32 <= a.N) {
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(v[8 * qq + 0]) * gmul, __uint_as_float(v[8 * qq + 1]) * gmul);
+              o.y = pack_bf16x2(__uint_as_float(v[8 * qq + 2]) * gmul, __uint_as_float(v[8 * qq + 3]) * gmul);
+              o.z = pack_bf16x2(__uint_as_float(v[8 * qq + 4]) * gmul, __uint_as_float(v[8 * qq + 5]) * gmul);
+              o.w = pack_bf16x2(__uint_as_float(v[8 * qq + 6]) * gmul, __uint_as_float(v[8 * qq + 7]) * gmul);
+              *reinterpret_cast<uint4*>(yrow + nb + 8 * qq) = o;
+            }
+          } else {
+            for (int qq = 0; qq < 32; ++qq)
+              if (nb + qq < a.N) yrow[nb + qq] = uint16_t(f32_to_bf16_bits(__uint_as_float(v[qq]) * gmul));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
   }
   tc_fence_before();

@@ -255,6 +255,37 @@ W4A4Layout w4a4_layout(int64_t M, int64_t K) {
   return L;
 }
 
+// Persistent FP4 GEMM (scale tiles by TMA): one CTA per SM over 128 x 128 tiles.
+int launch_fp4_persistent(wq::Fp4Args& a, const uint8_t* wcodes, cudaStream_t st) {
+  using S = wq::Fp4PShape;
+  if (int e = make_tmap_2d(&a.tmB, wcodes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 2),
+                           wq::kFp4PBN, wq::kFp4BK / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+    return e;
+  if (int e = make_tmap_2d(&a.tmSB, a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 16),
+                           wq::kFp4PBN, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return e;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_fp4_persistent_kernel,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES),
+                           "fp4 persistent smem attribute"))
+      return e;
+    attr_set = true;
+  }
+  const int64_t tiles = ((a.N + wq::kFp4PBN - 1) / wq::kFp4PBN) * int64_t((a.M + wq::kGemmBM - 1) / wq::kGemmBM);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(std::min<int64_t>(tiles, 148)), 1, 1);
+  cfg.blockDim = dim3(S::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = S::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemm_fp4_persistent_kernel, a), "fp4 persistent gemm launch");
+}
+
 template <int BN>
 int launch_fp4_bn(wq::Fp4Args& a, const uint8_t* xcodes, const uint8_t* wcodes, cudaStream_t st) {
   using S = wq::Fp4Shape<BN>;
@@ -274,6 +305,7 @@ int launch_fp4_bn(wq::Fp4Args& a, const uint8_t* xcodes, const uint8_t* wcodes, 
                              16, CU_TENSOR_MAP_SWIZZLE_NONE))
       return e;
   }
+  if (a.sf_tma) return launch_fp4_persistent(a, wcodes, st);
   static bool attr_set = false;
   if (!attr_set) {
     if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_fp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
