@@ -230,6 +230,15 @@ int wq_linear_nvfp4_w4a4_noalloc(const uint16_t* X, int64_t M, int64_t N, int64_
                                  const float* global_scale, const float* act_inv_s, uint16_t* Y,
                                  void* stream);
 
+/* wq_selftest_timeout -- exercises the failure path of the bounded waits on
+ * the GPU without a fault: launches one kernel whose single thread waits on
+ * an mbarrier that nothing arrives on.  After the 2 s limit the wait gives
+ * up, records a timeout in the device error word, stores 0 into
+ * *waited_ok (device int; 1 would mean the wait completed) and the kernel
+ * returns.  A following wq_device_error reports WQ_ERR_TIMEOUT and clears the
+ * word.  The pages have no counterpart: it is a test hook of this library. */
+int wq_selftest_timeout(int* waited_ok, void* stream);
+
 /* Synchronizes `stream`, then reads and clears the device error word of the
  * current GPU.  WQ_OK if no kernel reported a problem since the last call,
  * WQ_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the kernel then

@@ -42,6 +42,7 @@ SIGNATURES = {
     "wq_linear_nvfp4": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "wq_linear_nvfp4_w4a4_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P]),
     "wq_linear_group": (_I, [_P, _I, _I64, _P]),
+    "wq_selftest_timeout": (_I, [_P, _P]),
     "wq_device_error": (_I, [_P]),
 }
 
@@ -313,6 +314,16 @@ def wq_linear_group(calls, group=None):
     items it serves)."""
     arr, M = group if group is not None else make_group(calls)
     _check(load().wq_linear_group(ctypes.cast(arr, ctypes.c_void_p), len(arr), M, _stream()), "wq_linear_group")
+
+
+def wq_selftest_timeout() -> int:
+    """Launch the self-test whose bounded device wait runs out (about 2 s); returns the
+    kernel's waited_ok flag (0: the wait gave up as designed). Read the outcome with
+    wq_device_error(), which then raises WQError with WQ_ERR_TIMEOUT."""
+    flag = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _check(load().wq_selftest_timeout(_ptr(flag), _stream()), "wq_selftest_timeout")
+    torch.cuda.synchronize()
+    return int(flag.item())
 
 
 def wq_device_error() -> int:

@@ -879,6 +879,12 @@ int wq_linear_nvfp4_w4a4_noalloc(const uint16_t* X, int64_t M, int64_t N, int64_
   return gemm_bn(M, N) == 256 ? launch_fp4_bn<256>(f, xcodes, codes, st) : launch_fp4_bn<128>(f, xcodes, codes, st);
 }
 
+int wq_selftest_timeout(int* waited_ok, void* stream) {
+  REQUIRE_PTR(waited_ok);
+  wq::selftest_timeout_kernel<<<1, 32, 0, as_stream(stream)>>>(waited_ok);
+  return launched("selftest_timeout launch");
+}
+
 int wq_device_error(void* stream) {
   cudaStream_t st = as_stream(stream);
   if (int e = cuda_check(cudaStreamSynchronize(st), "stream synchronize")) return e;

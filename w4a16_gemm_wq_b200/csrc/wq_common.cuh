@@ -155,4 +155,16 @@ __device__ __forceinline__ uint4 ldg_v4(const void* p) {
   return v;
 }
 
+// Self-test of the failure path: one thread waits on an mbarrier that nothing
+// arrives on.  The bounded wait runs out after kWaitLimitNs, sets
+// ERR_TIMEOUT_PIPE in the device error word and returns; nothing faults or hangs.
+__global__ void selftest_timeout_kernel(int* waited_ok) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    *waited_ok = mbar_wait(&bar, 0, ERR_TIMEOUT_PIPE, nullptr) ? 1 : 0;
+  }
+}
+
 }  // namespace wq
