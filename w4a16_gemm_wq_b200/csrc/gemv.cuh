@@ -167,9 +167,9 @@ __device__ __forceinline__ void load_x32(const uint16_t* __restrict__ xrow, cons
   *sum = s;
 }
 
-template <int FMT, int MT>
+// R: weight rows per warp (4; 2 gives small-N problems twice the CTAs).
+template <int FMT, int MT, int R = kGemvRows>
 __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a) {
-  constexpr int R = kGemvRows;
   __shared__ float part[kGemvWarps * R * MT];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n0 = (blockIdx.x * kGemvWarps + warp) * R;

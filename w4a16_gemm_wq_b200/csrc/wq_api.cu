@@ -75,14 +75,18 @@ cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 int launched(const char* what) { return cuda_check(cudaGetLastError(), what); }
 
 // ---------------------------------------------------------------- GEMV launch
-template <int FMT, int MT>
-int launch_gemv_mt(const wq::GemvArgs& a0, cudaStream_t st) {
+// Launch shape of the CUDA-core GEMV, measured per weight kind on the decode
+// shapes: INT4 at N <= 2048 takes 2 rows per warp (twice the CTAs); INT4 with
+// long K (>= 8 k-iterations) targets 4 CTAs per SM through more split-K, the
+// rest 2 CTAs per SM.
+template <int FMT, int MT, int R>
+int launch_gemv_mtr(const wq::GemvArgs& a0, cudaStream_t st, int ctas_per_sm) {
   wq::GemvArgs a = a0;
-  const int rows_per_cta = wq::kGemvWarps * wq::kGemvRows;
+  const int rows_per_cta = wq::kGemvWarps * R;
   const int gx = (a.N + rows_per_cta - 1) / rows_per_cta;
   const int gz = (a.M + MT - 1) / MT;
   const int iters = (a.K + wq::kGemvKPerIter - 1) / wq::kGemvKPerIter;
-  int splits = (2 * 148 + gx * gz - 1) / (gx * gz);
+  int splits = (ctas_per_sm * 148 + gx * gz - 1) / (gx * gz);
   splits = std::max(1, std::min({splits, wq::kGemvMaxSplits, iters}));
   a.iters_per_split = (iters + splits - 1) / splits;
   splits = (iters + a.iters_per_split - 1) / a.iters_per_split;
@@ -108,7 +112,17 @@ int launch_gemv_mt(const wq::GemvArgs& a0, cudaStream_t st) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemv_kernel<FMT, MT>, a), "gemv launch");
+  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemv_kernel<FMT, MT, R>, a), "gemv launch");
+}
+
+template <int FMT, int MT>
+int launch_gemv_mt(const wq::GemvArgs& a, cudaStream_t st) {
+  const int iters = (a.K + wq::kGemvKPerIter - 1) / wq::kGemvKPerIter;
+  if (FMT == wq::FMT_INT4 && MT == 1) {
+    if (a.N <= 2048 && iters < 8) return launch_gemv_mtr<FMT, MT, 2>(a, st, 2);
+    return launch_gemv_mtr<FMT, MT, wq::kGemvRows>(a, st, iters >= 8 ? 4 : 2);
+  }
+  return launch_gemv_mtr<FMT, MT, wq::kGemvRows>(a, st, 2);
 }
 
 template <int FMT>
