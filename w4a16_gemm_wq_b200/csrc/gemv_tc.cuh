@@ -1,6 +1,6 @@
 // gemv_tc.cuh -- decode GEMV (M = 1 or 2 activation rows) on the tensor
-// cores, for one quantized Linear or a list of independent ones of the same
-// kind in a single launch.
+// cores, for one quantized Linear or a list of independent ones (INT4 g64,
+// INT4 g128 and NVFP4 mixed) in a single launch.
 //
 // Decode reads every packed weight once per token ("quantization primer"
 // section 13: memory-bound decode is where 4-bit weights pay off).  On B200 an
@@ -71,6 +71,7 @@ struct TcItem {
   uint16_t* Y;              // bf16 [M, N]
   int N, K;
   int xslot;                // staged activation vector
+  int kind;                 // TcKind of the weights
   int nrb, steps;           // row blocks, steps per row block (K / 128)
   int rb0;                  // first row block in the launch's row-block sequence
 };
@@ -312,14 +313,12 @@ __device__ __forceinline__ TcPos tc_pos(const TcArgs& a, int R0, int R1, int t) 
   }
 }
 
+// The work of one CTA whose row blocks all hold weights of kind KIND.
 template <int M, int KIND>
-__global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_constant__ TcArgs a) {
+__device__ __forceinline__ void gemv_tc_cta(const TcArgs& a, uint8_t* tc_smem, float* spart, unsigned* sctr,
+                                            int* xoff) {
   static_assert(M == 1 || M == 2, "M is 1 or 2");
   static_assert(KIND != TC_NVFP4_COLS || M == 1, "NVFP4 block columns need all 8 B columns");
-  extern __shared__ __align__(16) uint8_t tc_smem[];
-  __shared__ float spart[kTcWarps * 2 * kTcRows * M];  // partials of row blocks split over warps
-  __shared__ unsigned sctr[kTcWarps];                   // their arrival counters (by first piece's warp)
-  __shared__ int xoff[kTcMaxX];                         // byte offset of each staged vector, -1 if unused
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int R0 = a.bounds[blockIdx.x], R1 = a.bounds[blockIdx.x + 1];
@@ -578,6 +577,27 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
         ++C.j;
       }
     }
+  }
+}
+
+// One launch for a group of any weight kinds: every CTA's row blocks are of
+// one kind (the host splits the CTAs over the kinds by bytes), and the CTA
+// runs that kind's code.
+template <int M>
+__global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_constant__ TcArgs a) {
+  extern __shared__ __align__(16) uint8_t tc_smem[];
+  __shared__ float spart[kTcWarps * 2 * kTcRows * M];  // partials of row blocks split over warps
+  __shared__ unsigned sctr[kTcWarps];                   // their arrival counters (by first piece's warp)
+  __shared__ int xoff[kTcMaxX];                         // byte offset of each staged vector, -1 if unused
+  const int kind = a.items[tc_item_of_rb(a, a.bounds[blockIdx.x])].kind;
+  if (kind == TC_INT4_G64) {
+    gemv_tc_cta<M, TC_INT4_G64>(a, tc_smem, spart, sctr, xoff);
+  } else if (kind == TC_INT4_G128) {
+    gemv_tc_cta<M, TC_INT4_G128>(a, tc_smem, spart, sctr, xoff);
+  } else if constexpr (M == 1) {
+    gemv_tc_cta<M, TC_NVFP4_COLS>(a, tc_smem, spart, sctr, xoff);
+  } else {
+    gemv_tc_cta<M, TC_NVFP4_MUL>(a, tc_smem, spart, sctr, xoff);
   }
 }
 

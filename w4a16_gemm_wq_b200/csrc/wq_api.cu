@@ -390,59 +390,107 @@ int tc_kind(const TcCall& c, int64_t M) {
   return M == 1 ? wq::TC_NVFP4_COLS : wq::TC_NVFP4_MUL;
 }
 
-// Builds one launch over calls of one kind: items with their row-block
-// offsets, distinct activation vectors, the CTAs' row-block ranges (balanced
-// by bytes) and the staged activation bytes the busiest CTA needs.  Returns
-// false when the calls do not fit one launch.
-bool build_tc_args(const TcCall* calls, int count, int64_t M, wq::TcArgs* g, int* nctas, size_t* smem) {
+// Builds one launch over calls (each with its kind; all kinds in one launch):
+// items ordered by kind with their row-block offsets, distinct activation
+// vectors, the CTAs split over the kinds by bytes and, within a kind, into
+// byte-balanced contiguous row-block ranges, and the staged activation bytes
+// the busiest CTA needs.  Returns false when the calls do not fit one launch.
+bool build_tc_args(const TcCall* calls, const int* kinds, int count, int64_t M, wq::TcArgs* g, int* nctas,
+                   size_t* smem) {
   if (count < 1 || count > wq::kTcMaxItems) return false;
   memset(g, 0, sizeof(*g));
   g->n_items = count;
   int rb = 0;
   std::vector<double> cost;
-  for (int i = 0; i < count; ++i) {
-    const TcCall& c = calls[i];
-    wq::TcItem& d = g->items[i];
-    d.packed = static_cast<const uint8_t*>(c.packed);
-    d.scales = c.scales;
-    d.zeros = c.zeros;
-    d.bscale = c.bscale;
-    d.gscale = c.gscale;
-    d.Y = c.Y;
-    d.N = int(c.N);
-    d.K = int(c.K);
-    d.nrb = int((c.N + wq::kTcRows - 1) / wq::kTcRows);
-    d.steps = int(c.K / wq::kTcStepK);
-    d.rb0 = rb;
-    const int xg = c.fmt == wq::FMT_INT4 ? c.group_size : 0;
-    int slot = -1;
-    for (int v = 0; v < g->n_x; ++v)
-      if (g->xs[v].X == c.X && g->xs[v].K == d.K && g->xs[v].inv_s == c.inv_s && g->xs[v].g == xg) slot = v;
-    if (slot < 0) {
-      if (g->n_x == wq::kTcMaxX) return false;
-      slot = g->n_x++;
-      g->xs[slot] = wq::TcX{c.X, c.inv_s, d.K, xg};
+  double kcost[4] = {0, 0, 0, 0};
+  int krb[4] = {0, 0, 0, 0};
+  int n = 0;
+  for (int kind = 0; kind < 4; ++kind) {
+    for (int i = 0; i < count; ++i) {
+      if (kinds[i] != kind) continue;
+      const TcCall& c = calls[i];
+      wq::TcItem& d = g->items[n++];
+      d.packed = static_cast<const uint8_t*>(c.packed);
+      d.scales = c.scales;
+      d.zeros = c.zeros;
+      d.bscale = c.bscale;
+      d.gscale = c.gscale;
+      d.Y = c.Y;
+      d.N = int(c.N);
+      d.K = int(c.K);
+      d.kind = kind;
+      d.nrb = int((c.N + wq::kTcRows - 1) / wq::kTcRows);
+      d.steps = int(c.K / wq::kTcStepK);
+      d.rb0 = rb;
+      const int xg = c.fmt == wq::FMT_INT4 ? c.group_size : 0;
+      int slot = -1;
+      for (int v = 0; v < g->n_x; ++v)
+        if (g->xs[v].X == c.X && g->xs[v].K == d.K && g->xs[v].inv_s == c.inv_s && g->xs[v].g == xg) slot = v;
+      if (slot < 0) {
+        if (g->n_x == wq::kTcMaxX) return false;
+        slot = g->n_x++;
+        g->xs[slot] = wq::TcX{c.X, c.inv_s, d.K, xg};
+      }
+      d.xslot = slot;
+      // bytes a row block streams (codes + scale data) plus a fixed allowance for its end
+      const double per = wq::kTcRows * (double(c.K / 2) + double(c.K / 64) * 2.5) + 1024.0;
+      for (int r = 0; r < d.nrb; ++r) cost.push_back(per);
+      kcost[kind] += per * d.nrb;
+      krb[kind] += d.nrb;
+      rb += d.nrb;
+      if (rb >= (1 << 28)) return false;
     }
-    d.xslot = slot;
-    // bytes a row block streams (codes + scale data) plus a fixed allowance for its end
-    const double per = wq::kTcRows * (double(c.K / 2) + double(c.K / 64) * 2.5) + 1024.0;
-    for (int r = 0; r < d.nrb; ++r) cost.push_back(per);
-    rb += d.nrb;
-    if (rb >= (1 << 28)) return false;
   }
-  const int B = std::min(wq::kTcMaxCtas, rb);
+  if (n != count) return false;
+  // CTAs per kind in proportion to bytes (at least one, at most one per row block)
   double total = 0;
-  for (double c : cost) total += c;
-  int b = 0;
-  double accum = 0;
-  g->bounds[0] = 0;
-  for (int r = 0; r < rb; ++r) {
-    accum += cost[size_t(r)];
-    const int left = rb - 1 - r, ctas_left = B - 1 - b;
-    if (b < B - 1 && (accum >= total * (b + 1) / B || left == ctas_left)) g->bounds[++b] = r + 1;
+  int kinds_used = 0;
+  for (int k = 0; k < 4; ++k) {
+    total += kcost[k];
+    kinds_used += krb[k] > 0;
   }
-  while (b < B - 1) g->bounds[++b] = rb;
-  g->bounds[B] = rb;
+  int kctas[4] = {0, 0, 0, 0};
+  int B = 0;
+  for (int k = 0; k < 4; ++k) {
+    if (!krb[k]) continue;
+    kctas[k] = std::min(krb[k], std::max(1, int(wq::kTcMaxCtas * kcost[k] / total)));
+    B += kctas[k];
+  }
+  while (B > wq::kTcMaxCtas) {  // rounding overflow: take from the largest
+    int kk = 0;
+    for (int k = 1; k < 4; ++k)
+      if (kctas[k] > kctas[kk]) kk = k;
+    --kctas[kk];
+    --B;
+  }
+  // contiguous byte-balanced ranges inside each kind's row blocks
+  int b = 0, r0 = 0;
+  g->bounds[0] = 0;
+  for (int k = 0; k < 4; ++k) {
+    if (!krb[k]) continue;
+    const int r1 = r0 + krb[k], Bk = kctas[k];
+    double accum = 0;
+    int made = 0;
+    for (int r = r0; r < r1 && made < Bk - 1; ++r) {
+      accum += cost[size_t(r)];
+      const int left = r1 - 1 - r, ctas_left = Bk - 1 - made;
+      if (accum >= kcost[k] * (made + 1) / Bk || left == ctas_left) {
+        g->bounds[++b] = r + 1;
+        ++made;
+      }
+    }
+    while (made < Bk - 1) {  // cannot happen with Bk <= row blocks; kept for safety
+      g->bounds[++b] = r1;
+      ++made;
+    }
+    g->bounds[++b] = r1;
+    r0 = r1;
+  }
+  // drop empty ranges (bounds must be strictly increasing)
+  int B2 = 0;
+  for (int i = 0; i < b; ++i)
+    if (g->bounds[i + 1] > g->bounds[i]) g->bounds[++B2] = g->bounds[i + 1];
+  B = B2;
   // staged activations of the busiest CTA
   const auto item_of = [&](int r) {
     int i = 0;
@@ -461,15 +509,16 @@ bool build_tc_args(const TcCall* calls, int count, int64_t M, wq::TcArgs* g, int
   *smem = xmax;
   if (*smem > size_t(wq::kTcMaxSmem)) return false;
   *nctas = B;
+  (void)kinds_used;
   return true;
 }
 
-template <int M, int KIND>
-int launch_tc_k(const wq::TcArgs& g, int nctas, size_t smem, cudaStream_t st) {
+template <int M>
+int launch_tc_m(const wq::TcArgs& g, int nctas, size_t smem, cudaStream_t st) {
   static bool attr_set = false;
   if (!attr_set) {
-    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemv_tc_kernel<M, KIND>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, wq::kTcMaxSmem),
+    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemv_tc_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                wq::kTcMaxSmem),
                            "gemv_tc smem attribute"))
       return e;
     attr_set = true;
@@ -484,48 +533,32 @@ int launch_tc_k(const wq::TcArgs& g, int nctas, size_t smem, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemv_tc_kernel<M, KIND>, g), "gemv_tc launch");
-}
-
-int launch_tc(const wq::TcArgs& g, int64_t M, int kind, int nctas, size_t smem, cudaStream_t st) {
-  if (M == 1) {
-    switch (kind) {
-      case wq::TC_INT4_G64: return launch_tc_k<1, wq::TC_INT4_G64>(g, nctas, smem, st);
-      case wq::TC_INT4_G128: return launch_tc_k<1, wq::TC_INT4_G128>(g, nctas, smem, st);
-      default: return launch_tc_k<1, wq::TC_NVFP4_COLS>(g, nctas, smem, st);
-    }
-  }
-  switch (kind) {
-    case wq::TC_INT4_G64: return launch_tc_k<2, wq::TC_INT4_G64>(g, nctas, smem, st);
-    case wq::TC_INT4_G128: return launch_tc_k<2, wq::TC_INT4_G128>(g, nctas, smem, st);
-    default: return launch_tc_k<2, wq::TC_NVFP4_MUL>(g, nctas, smem, st);
-  }
+  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemv_tc_kernel<M>, g), "gemv_tc launch");
 }
 
 // Runs calls (each with its kind, -1 = not served) through the tensor-core
-// decode GEMV, one launch per kind (<= kTcMaxItems calls each); done[i]
-// tells which calls it took.
+// decode GEMV: one launch for up to kTcMaxItems of them, all kinds together;
+// done[i] tells which calls it took.
 int run_tc(const TcCall* calls, const int* kinds, int count, int64_t M, cudaStream_t st, char* done) {
   static thread_local wq::TcArgs g;  // ~3 KB: keep it off the stack
   for (int i = 0; i < count; ++i) done[i] = 0;
-  for (int kind = 0; kind < 4; ++kind) {
-    for (int start = 0; start < count;) {
-      TcCall sub[wq::kTcMaxItems];
-      int idx[wq::kTcMaxItems];
-      int n = 0, i = start;
-      for (; i < count && n < wq::kTcMaxItems; ++i)
-        if (kinds[i] == kind) {
-          idx[n] = i;
-          sub[n++] = calls[i];
-        }
-      start = i;
-      if (n == 0) break;
-      int nctas = 0;
-      size_t smem = 0;
-      if (!build_tc_args(sub, n, M, &g, &nctas, &smem)) continue;
-      if (int e = launch_tc(g, M, kind, nctas, smem, st)) return e;
-      for (int j = 0; j < n; ++j) done[idx[j]] = 1;
-    }
+  for (int start = 0; start < count;) {
+    TcCall sub[wq::kTcMaxItems];
+    int sk[wq::kTcMaxItems], idx[wq::kTcMaxItems];
+    int n = 0, i = start;
+    for (; i < count && n < wq::kTcMaxItems; ++i)
+      if (kinds[i] >= 0) {
+        idx[n] = i;
+        sk[n] = kinds[i];
+        sub[n++] = calls[i];
+      }
+    start = i;
+    if (n == 0) break;
+    int nctas = 0;
+    size_t smem = 0;
+    if (!build_tc_args(sub, sk, n, M, &g, &nctas, &smem)) continue;
+    if (int e = (M == 1 ? launch_tc_m<1>(g, nctas, smem, st) : launch_tc_m<2>(g, nctas, smem, st))) return e;
+    for (int j = 0; j < n; ++j) done[idx[j]] = 1;
   }
   return WQ_OK;
 }
