@@ -38,6 +38,11 @@
 // order (bf16 -> f16 is exact in the normal range; x / s is rounded once),
 // INT4 with the group sums (of the f16 values the mma sees, so that the 1024 P
 // bias cancels exactly); the first weight loads are in flight meanwhile.
+// Lanes whose B column must stay empty (INT4 g64, NVFP4 at M = 1) read a
+// zeroed row with stride 0 instead of the activations, so the math has no
+// selects.  The host precomputes each CTA's first item, kind, step count and
+// activation vectors, so a CTA reaches the dependency wait after a few
+// parameter reads.  Code loads carry a 256-byte L2 prefetch hint.
 // Weights are prefetched into L2 before the programmatic-launch dependency
 // wait (L2 is the point of coherence, so this never yields stale data); every
 // load that feeds the math is issued after the wait.
@@ -59,6 +64,7 @@ constexpr int kTcStepK = 128;     // k per step
 constexpr int kTcWarps = 16;
 constexpr int kTcThreads = kTcWarps * 32;
 constexpr int kTcDepth = 3;       // steps in flight per warp (3 KB; 48 KB per SM)
+constexpr int kTcPrefetchFirst = 4;  // steps per warp brought into L2 before the dependency wait
 constexpr int kTcMaxCtas = 148;
 constexpr int kTcMaxSmem = 200 * 1024;
 
@@ -87,6 +93,8 @@ struct TcArgs {
   TcItem items[kTcMaxItems];
   TcX xs[kTcMaxX];
   int bounds[kTcMaxCtas + 1];  // row-block range of each CTA
+  uint32_t cta[kTcMaxCtas];    // per CTA: first item | last item << 5 | kind << 10 | steps << 12
+  uint8_t xused[kTcMaxCtas];   // per CTA: mask of the activation vectors its items read
   int n_items, n_x;
 };
 static_assert(sizeof(TcArgs) <= 4096, "kernel parameters must fit the 4 KB limit");
@@ -119,19 +127,12 @@ __device__ __forceinline__ void tc_mma(float (&d)[4], uint32_t a0, uint32_t a1, 
 }
 __device__ __forceinline__ uint4 tc_ld_stream(const void* p) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
 }
 __device__ __forceinline__ void tc_prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
-
-// Item holding global row block r (items are ordered by rb0).
-__device__ __forceinline__ int tc_item_of_rb(const TcArgs& a, int r) {
-  int i = 0;
-  while (i + 1 < a.n_items && a.items[i + 1].rb0 <= r) ++i;
-  return i;
-}
 
 // What one lane loads per step: 16 code bytes of rows g and g + 8 and their
 // scale data (INT4 G64: fp16 scale pair of groups 2j, 2j+1 + zero word;
@@ -295,10 +296,21 @@ __device__ __noinline__ void tc_flush_split(const float* v, int lane, int warp, 
   }
 }
 
+// L2 prefetch of steps [j, j + 4) of the 16 rows of row block rb: lane l takes
+// row l % 16 and the 128-byte line of steps j + 2 (l / 16), + 1 (as far as
+// the row block has steps).
+__device__ __forceinline__ void tc_prefetch_rows(const TcItem& I, int rb, int j, int lane) {
+  j += 2 * (lane >> 4);
+  if (rb < I.nrb && j < I.steps) {
+    const int n = min(rb * kTcRows + (lane & 15), I.N - 1);
+    tc_prefetch_l2(I.packed + int64_t(n) * (I.K >> 1) + 64 * j);
+  }
+}
+
 // Position (item, row block, step) of step t of the CTA's sequence over the
 // global row blocks [R0, R1).
-__device__ __forceinline__ TcPos tc_pos(const TcArgs& a, int R0, int R1, int t) {
-  TcPos p{tc_item_of_rb(a, R0), 0, 0};
+__device__ __forceinline__ TcPos tc_pos(const TcArgs& a, int i0, int R0, int R1, int t) {
+  TcPos p{i0, 0, 0};
   for (;; ++p.i) {
     const TcItem& I = a.items[p.i];
     const int r0 = max(R0, I.rb0), r1 = min(R1, I.rb0 + I.nrb);
@@ -316,35 +328,38 @@ __device__ __forceinline__ TcPos tc_pos(const TcArgs& a, int R0, int R1, int t) 
 // The work of one CTA whose row blocks all hold weights of kind KIND.
 template <int M, int KIND>
 __device__ __forceinline__ void gemv_tc_cta(const TcArgs& a, uint8_t* tc_smem, float* spart, unsigned* sctr,
-                                            int* xoff) {
+                                            int* xoff, const uint16_t* zrow) {
   static_assert(M == 1 || M == 2, "M is 1 or 2");
   static_assert(KIND != TC_NVFP4_COLS || M == 1, "NVFP4 block columns need all 8 B columns");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const int R0 = a.bounds[blockIdx.x], R1 = a.bounds[blockIdx.x + 1];
-  const int i0 = tc_item_of_rb(a, R0), i1 = tc_item_of_rb(a, R1 - 1);
-  int S = 0;  // steps of this CTA
-  for (int i = i0; i <= i1; ++i) {
-    const TcItem& I = a.items[i];
-    S += (min(R1, I.rb0 + I.nrb) - max(R0, I.rb0)) * I.steps;
-  }
+  const uint32_t info = a.cta[blockIdx.x];
+  const int i0 = int(info & 31u), S = int(info >> 12);  // first item, steps of this CTA
   const int Wc = min(kTcWarps, S);  // warps that share the steps (none empty)
   const int lo = warp < Wc ? (warp * S) / Wc : S, hi = warp < Wc ? ((warp + 1) * S) / Wc : S;
   if (threadIdx.x < kTcWarps) sctr[threadIdx.x] = 0;
+  if (threadIdx.x < 4) reinterpret_cast<uint4*>(const_cast<uint16_t*>(zrow))[threadIdx.x] = make_uint4(0, 0, 0, 0);
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // this warp's walk: loads run kTcDepth steps ahead of the math
-  TcPos L = tc_pos(a, R0, R1, lo);
+  TcPos L = tc_pos(a, i0, R0, R1, lo);
   TcPos C = L;
   TcLoadPtrs lp;
   tc_load_ptrs<KIND>(a.items[L.i], L.rb, g, c, lp);
   // warm L2 with the first steps while the previous grid drains (L2 is the
   // point of coherence: this never yields stale data; the loads come after the wait)
-  if (c == 0 && lo < hi)
-    for (int q = L.j; q < min(a.items[L.i].steps, L.j + kTcDepth); q += 2) {
-      tc_prefetch_l2(lp.clo + 64 * q);
-      tc_prefetch_l2(lp.chi + 64 * q);
+  if (lo < hi) {
+    const TcItem& I = a.items[L.i];
+    int rb = L.rb, j = L.j;
+    for (int t = 0; t < min(kTcPrefetchFirst, hi - lo); t += 4) {  // may run into the next row block
+      tc_prefetch_rows(I, rb, j, lane);
+      if ((j += 4) >= I.steps) {
+        j = 0;
+        ++rb;
+      }
     }
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   int lsteps = a.items[L.i].steps;
@@ -371,8 +386,7 @@ __device__ __forceinline__ void gemv_tc_cta(const TcArgs& a, uint8_t* tc_smem, f
 
   // ---- stage this CTA's activation vectors (f16, fragment order, INT4 group sums)
   if (threadIdx.x == 0) {
-    uint32_t used = 0;
-    for (int i = i0; i <= i1; ++i) used |= 1u << a.items[i].xslot;
+    const uint32_t used = a.xused[blockIdx.x];
     int off = 0;
     for (int v = 0; v < kTcMaxX; ++v) {
       xoff[v] = -1;
@@ -444,11 +458,13 @@ __device__ __forceinline__ void gemv_tc_cta(const TcArgs& a, uint8_t* tc_smem, f
   __syncthreads();
   if (lo >= hi) return;
 
-  // per-item compute state: this lane's B source, whether it feeds words 0-1 /
-  // 2-3 at all, the INT4 group sums
+  // per-item compute state: this lane's B sources for words 0-1 / 2-3 and
+  // their stride per step (0 on the zeroed row when the lane's column must stay
+  // empty), the INT4 group sums
   const uint16_t* xa = nullptr;
+  const uint16_t* xb = nullptr;
+  int xsa = 0, xsb = 0;
   const float2* sums = nullptr;
-  bool va = false, vb = false;
   int csteps = 0;
   float gmul = 1.f;
   const auto compute_enter = [&]() {
@@ -457,6 +473,7 @@ __device__ __forceinline__ void gemv_tc_cta(const TcArgs& a, uint8_t* tc_smem, f
     csteps = I.steps;
     sums = reinterpret_cast<const float2*>(xbase + M * I.K * 2);
     gmul = (KIND == TC_NVFP4_COLS || KIND == TC_NVFP4_MUL) ? __ldg(I.gscale) : 1.f;
+    bool va = true, vb = true;
     int m = 0;
     if (KIND == TC_INT4_G64) {  // column 2m + (c >= 2)
       const int d = g - (c >> 1);
@@ -465,11 +482,14 @@ __device__ __forceinline__ void gemv_tc_cta(const TcArgs& a, uint8_t* tc_smem, f
     } else if (KIND == TC_NVFP4_COLS) {  // column = block 2c + (word >= 2)
       va = g == 2 * c;
       vb = g == 2 * c + 1;
-    } else {  // column m
-      va = vb = g < M;
-      m = va ? g : 0;
+    } else {  // column m; the outputs of the other columns are never read
+      m = g < M ? g : 0;
     }
-    xa = reinterpret_cast<const uint16_t*>(xbase) + m * I.K + 32 * c;
+    const uint16_t* xl = reinterpret_cast<const uint16_t*>(xbase) + m * I.K + 32 * c;
+    xa = va ? xl : zrow;
+    xb = vb ? xl : zrow;
+    xsa = va ? kTcStepK : 0;
+    xsb = vb ? kTcStepK : 0;
   };
   compute_enter();
 
@@ -482,7 +502,8 @@ __device__ __forceinline__ void gemv_tc_cta(const TcArgs& a, uint8_t* tc_smem, f
       // ---------------------------------------------------------- math of step s
       {
         const TcEntry& e = R[u];
-        const uint16_t* xs = xa + C.j * kTcStepK;
+        const uint16_t* xsA = xa + C.j * xsa;
+        const uint16_t* xsB = xb + C.j * xsb;
         float d[4] = {0.f, 0.f, 0.f, 0.f}, f[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t sbl = 0, sbh = 0;
         if (KIND == TC_NVFP4_MUL) {
@@ -491,8 +512,7 @@ __device__ __forceinline__ void gemv_tc_cta(const TcArgs& a, uint8_t* tc_smem, f
         }
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          const bool v = w < 2 ? va : vb;
-          const uint4 b = v ? *reinterpret_cast<const uint4*>(xs + 8 * w) : make_uint4(0, 0, 0, 0);
+          const uint4 b = *reinterpret_cast<const uint4*>((w < 2 ? xsA : xsB) + 8 * w);
           const uint32_t wl = w == 0 ? e.lo.x : w == 1 ? e.lo.y : w == 2 ? e.lo.z : e.lo.w;
           const uint32_t wh = w == 0 ? e.hi.x : w == 1 ? e.hi.y : w == 2 ? e.hi.z : e.hi.w;
           uint32_t l0, l2, l0n, l2n, h0, h2, h0n, h2n;
@@ -589,15 +609,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemv_tc_kernel(const __grid_con
   __shared__ float spart[kTcWarps * 2 * kTcRows * M];  // partials of row blocks split over warps
   __shared__ unsigned sctr[kTcWarps];                   // their arrival counters (by first piece's warp)
   __shared__ int xoff[kTcMaxX];                         // byte offset of each staged vector, -1 if unused
-  const int kind = a.items[tc_item_of_rb(a, a.bounds[blockIdx.x])].kind;
+  __shared__ __align__(16) uint16_t zrow[32];           // B source of lanes whose column stays empty
+  const int kind = int((a.cta[blockIdx.x] >> 10) & 3u);
   if (kind == TC_INT4_G64) {
-    gemv_tc_cta<M, TC_INT4_G64>(a, tc_smem, spart, sctr, xoff);
+    gemv_tc_cta<M, TC_INT4_G64>(a, tc_smem, spart, sctr, xoff, zrow);
   } else if (kind == TC_INT4_G128) {
-    gemv_tc_cta<M, TC_INT4_G128>(a, tc_smem, spart, sctr, xoff);
+    gemv_tc_cta<M, TC_INT4_G128>(a, tc_smem, spart, sctr, xoff, zrow);
   } else if constexpr (M == 1) {
-    gemv_tc_cta<M, TC_NVFP4_COLS>(a, tc_smem, spart, sctr, xoff);
+    gemv_tc_cta<M, TC_NVFP4_COLS>(a, tc_smem, spart, sctr, xoff, zrow);
   } else {
-    gemv_tc_cta<M, TC_NVFP4_MUL>(a, tc_smem, spart, sctr, xoff);
+    gemv_tc_cta<M, TC_NVFP4_MUL>(a, tc_smem, spart, sctr, xoff, zrow);
   }
 }
 

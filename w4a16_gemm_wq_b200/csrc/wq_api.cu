@@ -432,8 +432,10 @@ bool build_tc_args(const TcCall* calls, const int* kinds, int count, int64_t M, 
         g->xs[slot] = wq::TcX{c.X, c.inv_s, d.K, xg};
       }
       d.xslot = slot;
-      // bytes a row block streams (codes + scale data) plus a fixed allowance for its end
-      const double per = wq::kTcRows * (double(c.K / 2) + double(c.K / 64) * 2.5) + 1024.0;
+      // time of a row block: its steps (one 1 KB code tile each, at the kind's
+      // measured cost per step relative to INT4 g128) plus an allowance for its end
+      static const double kStepCost[4] = {1.04, 1.0, 0.975, 1.0};
+      const double per = double(d.steps) * 1024.0 * kStepCost[kind] + 1024.0;
       for (int r = 0; r < d.nrb; ++r) cost.push_back(per);
       kcost[kind] += per * d.nrb;
       krb[kind] += d.nrb;
@@ -491,7 +493,8 @@ bool build_tc_args(const TcCall* calls, const int* kinds, int count, int64_t M, 
   for (int i = 0; i < b; ++i)
     if (g->bounds[i + 1] > g->bounds[i]) g->bounds[++B2] = g->bounds[i + 1];
   B = B2;
-  // staged activations of the busiest CTA
+  // per CTA: first / last item, kind, steps, activation vectors; the staged
+  // activations of the busiest CTA
   const auto item_of = [&](int r) {
     int i = 0;
     while (i + 1 < count && g->items[i + 1].rb0 <= r) ++i;
@@ -499,8 +502,18 @@ bool build_tc_args(const TcCall* calls, const int* kinds, int count, int64_t M, 
   };
   size_t xmax = 0;
   for (int cb = 0; cb < B; ++cb) {
+    const int R0 = g->bounds[cb], R1 = g->bounds[cb + 1];
+    const int i0 = item_of(R0), i1 = item_of(R1 - 1);
     uint32_t used = 0;
-    for (int i = item_of(g->bounds[cb]); i <= item_of(g->bounds[cb + 1] - 1); ++i) used |= 1u << g->items[i].xslot;
+    int64_t steps = 0;
+    for (int i = i0; i <= i1; ++i) {
+      const wq::TcItem& I = g->items[i];
+      used |= 1u << I.xslot;
+      steps += int64_t(std::min(R1, I.rb0 + I.nrb) - std::max(R0, I.rb0)) * I.steps;
+    }
+    if (steps >= (int64_t(1) << 20) || g->items[i0].kind != g->items[i1].kind) return false;
+    g->cta[cb] = uint32_t(i0) | uint32_t(i1) << 5 | uint32_t(g->items[i0].kind) << 10 | uint32_t(steps) << 12;
+    g->xused[cb] = uint8_t(used);
     size_t x = 0;
     for (int v = 0; v < g->n_x; ++v)
       if ((used >> v) & 1) x += size_t(wq::tc_x_bytes(g->xs[v].K, g->xs[v].g, int(M)));
