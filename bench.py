@@ -372,7 +372,8 @@ def run_ours(args):
     if not args.no_aux:
         out["quantize"] = {"workload": "7 projections of one block: INT4 g64 with AWQ scale, NVFP4",
                            "results": quant_measure(wq, synth, torch, dev, peaks)}
-        out["awq_search"] = {"workload": "7 projections, 512 Student-t calibration tokens, 20 alphas, G=64",
+        out["awq_search"] = {"workload": "7 projections, 512 Student-t calibration tokens, 20 alphas, G=64; "
+                                         "shared_s: one s for q/k/v and one for gate/up (stacked rows)",
                              "results": awq_measure(wq, synth, torch, dev, peaks)}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
@@ -497,9 +498,30 @@ def awq_measure(wq, synth, torch, dev, peaks, T=512):
         per[name] = round(sec * 1e3, 3)
         tot_s += sec
         tot_flop += flop
+    # one s shared by the matrices that consume one normalised input (folded into
+    # that RMSNorm): q/k/v (N = 2048 + 256 + 256) and gate/up (N = 2 x 11008)
+    shared = {}
+    by_name = {name: (K, N) for name, K, N in synth.PROJECTIONS}
+    for gname, names in (("qkv", ("q_proj", "k_proj", "v_proj")), ("gate_up", ("gate_proj", "up_proj"))):
+        K = by_name[names[0]][0]
+        Ws = [synth.weight(by_name[n][1], K, seed=synth.layer_seed(3, K + by_name[n][1] + j), device=dev)
+              for j, n in enumerate(names)]
+        X = synth.activations_student_t(T, K, seed=synth.layer_seed(3, K), device=dev)
+        wq.awq_search_scale_shared(Ws, alphas, 64, X=X)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        wq.awq_search_scale_shared(Ws, alphas, 64, X=X)
+        b.record()
+        torch.cuda.synchronize()
+        sec = a.elapsed_time(b) * 1e-3
+        Nt = sum(W.shape[0] for W in Ws)
+        flop = 2.0 * T * Nt * (2 * K) * len(synth.ALPHA_GRID)
+        shared[gname] = {"N": Nt, "K": K, "ms": round(sec * 1e3, 3), "loss_gemm_TFLOP/s": round(flop / sec / 1e12, 1)}
     return {"ms_per_projection": per, "ms_total": round(tot_s * 1e3, 3),
             "loss_gemm_TFLOP/s": round(tot_flop / tot_s / 1e12, 1),
-            "frac_of_bf16_sustained": round(tot_flop / tot_s / 1e12 / peaks["bf16_sustained"], 4)}
+            "frac_of_bf16_sustained": round(tot_flop / tot_s / 1e12 / peaks["bf16_sustained"], 4),
+            "shared_s": shared}
 
 
 # ---------------------------------------------------------------- oracle arm

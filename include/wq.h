@@ -148,6 +148,26 @@ int awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X,
                      float* s_out, float* loss_out, int* best_idx, void* ws, size_t ws_bytes,
                      void* stream);
 
+/* awq_search_scale_shared -- the same grid search for several weight
+ * matrices that consume one input and therefore share one s ("Lance-Quant"
+ * section "量化应用：网格搜索与分组策略": the AWQ scale of a norm and the
+ * linear layers consuming it is folded into that RMSNorm, so q/k/v share one
+ * s and gate/up share one; section "v2改进" notes o/down cannot).  The loss
+ * of alpha_i is the loss of the stacked matrix [W_0; W_1; ...] (N = sum of
+ * Ns rows): the sum of the matrices' losses under the one s.
+ *   Ws       host array of n_mats (1..64) device pointers, bf16 [Ns[p], K],
+ *            16-byte aligned
+ *   Ns       host array of the row counts
+ *   ws_bytes from awq_search_workspace_size(sum of Ns, K, T, n_alpha, G)
+ * Every other argument and the errors are those of awq_search_scale; the
+ * chosen s then quantizes each matrix (wq_quantize_int4 with scale_s = s), or
+ * the stacked matrix once, whose pack is the stack of the matrices' packs
+ * (rows are quantized independently), for one fused linear over N rows. */
+int awq_search_scale_shared(const uint16_t* const* Ws, const int64_t* Ns, int n_mats, int64_t K,
+                            const uint16_t* X, int64_t T, const float* act_mean, const float* alphas,
+                            int n_alpha, int group_size, float* s_out, float* loss_out, int* best_idx,
+                            void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- stage 2: quantized Linear
  * wq_linear_int4 -- Y = (X * act_inv_s) * dequant(Wq)^T, bf16 in, fp32
  * accumulate, bf16 out ("quantization primer" sections 4 and 13).

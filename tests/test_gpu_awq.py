@@ -104,3 +104,45 @@ def test_config3_full_shapes_two_alphas(lib, name, K, N):
         ref = float(np.sum(y * y))
         assert abs(losses[i] - ref) <= LOSS_RTOL * ref, (i, losses[i], ref)
     assert _ulps(s, np.power(a, float(ALPHAS[best])).astype(np.float32)) <= 4
+
+
+@pytest.mark.parametrize("G", [64, 128])
+@pytest.mark.parametrize("proxy", [False, True])
+def test_shared_scale_qkv_like(lib, G, proxy):
+    # one s for three matrices that consume one input (q/k/v-like row counts, one of
+    # them ragged): losses, choice and s against the oracle's search over the stacked
+    # rows; each matrix's pack with that s bit-exact; the stacked pack is the stack of packs
+    K, T = 512, 96
+    Ns = (80, 24, 17)
+    Ws = [synth.weight(n, K, seed=50 + i, outlier_frac=0.02) for i, n in enumerate(Ns)]
+    X = None if proxy else synth.activations_student_t(T, K, seed=50)
+    am = synth.act_mean_lognormal(K, seed=50).numpy() if proxy else None
+    s, losses, best = lib.awq_search_scale_shared(
+        [W.cuda() for W in Ws], torch.tensor(ALPHAS).cuda(), G, X=None if X is None else X.cuda(),
+        act_mean=None if am is None else torch.tensor(am).cuda())
+    torch.cuda.synchronize()
+    s, losses, best = s.cpu().numpy(), losses.cpu().numpy().astype(np.float64), int(best.cpu()[0])
+    s_ref, losses_ref, best_ref = oracle.awq_search(torch.cat(Ws), G, ALPHAS, X=X, act_mean=am)
+    np.testing.assert_allclose(losses, losses_ref, rtol=LOSS_RTOL)
+    assert best == int(np.argmin(losses))
+    _check_choice(losses_ref, best, best_ref)
+    a = oracle.awq_mean_abs(X) if X is not None else np.maximum(am.astype(np.float64), 1e-4)
+    assert _ulps(s, np.power(a, float(ALPHAS[best])).astype(np.float32)) <= 4
+    st = torch.tensor(s).cuda()
+    stacked = lib.wq_quantize_int4(torch.cat(Ws).cuda(), G, 1, st)
+    packs = [lib.wq_quantize_int4(W.cuda(), G, 1, st) for W in Ws]
+    torch.cuda.synchronize()
+    for W, p in zip(Ws, packs):
+        ref = oracle.quantize_int4(W, G, s=s)
+        np.testing.assert_array_equal(bits(p.qweight), ref["qweight"])
+        np.testing.assert_array_equal(bits(p.scales), ref["scales"])
+        np.testing.assert_array_equal(bits(p.zeros), ref["zeros"])
+    for name in ("qweight", "scales", "zeros"):
+        np.testing.assert_array_equal(bits(getattr(stacked, name)),
+                                      np.concatenate([bits(getattr(p, name)) for p in packs]))
+
+
+def test_shared_scale_rejects_mismatched_k(lib):
+    Ws = [synth.weight(16, 256, seed=1).cuda(), synth.weight(16, 512, seed=2).cuda()]
+    with pytest.raises(ValueError):
+        lib.awq_search_scale_shared(Ws, torch.tensor(ALPHAS).cuda(), 64, act_mean=torch.ones(256).cuda())

@@ -399,3 +399,19 @@ def test_awq_helps_on_outlier_channels():
     s, losses, best = oracle.awq_search(W, G, ALPHAS, X=X)
     assert best > 0 and losses[best] < losses[0]
     assert d["W"].shape == (512, 512)
+
+
+def test_awq_shared_scale_is_the_search_over_stacked_rows():
+    # Matrices that consume one normalised input (q/k/v, gate/up) share one s, since
+    # the scale is folded into that RMSNorm ("Lance-Quant", section 量化应用): the loss
+    # of the stack [W_0; W_1; W_2] under s is the sum of the matrices' losses under the
+    # same s, for the token loss and for the diagonal proxy alike.
+    T, K, G = 32, 256, 64
+    Ws = [synth.weight(n, K, seed=40 + i, outlier_frac=0.02) for i, n in enumerate((32, 8, 8))]
+    X = synth.activations_student_t(T, K, seed=40)
+    a = synth.act_mean_lognormal(K, seed=40).numpy()
+    for kw in ({"X": X}, {"act_mean": a}):
+        parts = np.sum([oracle.awq_search(W, G, ALPHAS, **kw)[1] for W in Ws], axis=0)
+        s, shared, best = oracle.awq_search(torch.cat(Ws), G, ALPHAS, **kw)
+        np.testing.assert_allclose(shared, parts, rtol=1e-12)
+        assert best == int(np.argmin(parts))

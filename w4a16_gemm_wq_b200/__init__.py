@@ -8,8 +8,8 @@ library's CUDA kernels.  There is no CPU fallback: if the library cannot be
 loaded every call raises.
 
 Functions carry the C names:
-    wq_quantize_int4, wq_quantize_nvfp4, awq_search_scale,
-    wq_linear_int4, wq_linear_nvfp4, wq_device_error
+    wq_quantize_int4, wq_quantize_nvfp4, awq_search_scale, awq_search_scale_shared,
+    wq_linear_int4, wq_linear_nvfp4, wq_linear_group, wq_device_error
 """
 from __future__ import annotations
 
@@ -38,6 +38,7 @@ SIGNATURES = {
     "wq_quantize_int4": (_I, [_P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
     "wq_quantize_nvfp4": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "awq_search_scale": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P]),
+    "awq_search_scale_shared": (_I, [_P, _P, _I, _I64, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "wq_linear_int4": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _I, _P, _P, _P, _SZ, _P]),
     "wq_linear_nvfp4": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "wq_linear_nvfp4_w4a4_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P]),
@@ -212,6 +213,45 @@ def awq_search_scale(W: torch.Tensor, alphas: torch.Tensor, group_size: int = 64
     best = torch.empty(1, dtype=torch.int32, device=W.device)
     _check(lib.awq_search_scale(_ptr(W), N, K, _ptr(X), T, _ptr(am), _ptr(alphas), n_alpha, group_size, _ptr(s),
                                 _ptr(losses), _ptr(best), _ptr(ws), b.value, _stream()), "awq_search_scale")
+    return s, losses, best
+
+
+def awq_search_scale_shared(Ws: list, alphas: torch.Tensor, group_size: int = 64, X: torch.Tensor | None = None,
+                            act_mean: torch.Tensor | None = None):
+    """One AWQ scale for several weights that consume the same input (q/k/v,
+    gate/up): the loss is taken over their stacked rows.  Returns (s fp32 [K],
+    losses fp32 [n_alpha], best int32 [1]) as device tensors."""
+    if not Ws:
+        raise ValueError("need at least one weight matrix")
+    for i, W in enumerate(Ws):
+        _dev(W, f"Ws[{i}]", torch.bfloat16)
+    K = Ws[0].shape[1]
+    if any(W.dim() != 2 or W.shape[1] != K for W in Ws):
+        raise ValueError("every weight must be [N_i, K] with the same K")
+    T = 0
+    if X is not None:
+        _dev(X, "X", torch.bfloat16)
+        if X.dim() != 2 or X.shape[1] != K:
+            raise ValueError("X must be [T, K]")
+        T = X.shape[0]
+    am = _opt_f32(act_mean, "act_mean", K)
+    _dev(alphas, "alphas", torch.float32)
+    lib = load()
+    n_alpha = alphas.numel()
+    Ntot = sum(int(W.shape[0]) for W in Ws)
+    b = ctypes.c_size_t()
+    _check(lib.awq_search_workspace_size(Ntot, K, T, n_alpha, group_size, ctypes.byref(b)),
+           "awq_search_workspace_size")
+    ws = _workspace(b.value, Ws[0].device)
+    ptrs = (ctypes.c_void_p * len(Ws))(*[W.data_ptr() for W in Ws])
+    ns = (ctypes.c_int64 * len(Ws))(*[int(W.shape[0]) for W in Ws])
+    s = torch.empty(K, dtype=torch.float32, device=Ws[0].device)
+    losses = torch.empty(n_alpha, dtype=torch.float32, device=Ws[0].device)
+    best = torch.empty(1, dtype=torch.int32, device=Ws[0].device)
+    _check(lib.awq_search_scale_shared(ctypes.cast(ptrs, ctypes.c_void_p), ctypes.cast(ns, ctypes.c_void_p),
+                                       len(Ws), K, _ptr(X), T, _ptr(am), _ptr(alphas), n_alpha, group_size,
+                                       _ptr(s), _ptr(losses), _ptr(best), _ptr(ws), b.value, _stream()),
+           "awq_search_scale_shared")
     return s, losses, best
 
 

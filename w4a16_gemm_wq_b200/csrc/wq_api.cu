@@ -712,12 +712,21 @@ int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scal
   return nvfp4_quantize_launch(W, N, K, scale_s, codes, bscale, global_scale, as_stream(stream));
 }
 
-int awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t T, const float* act_mean,
-                     const float* alphas, int n_alpha, int group_size, float* s_out, float* loss_out, int* best_idx,
-                     void* ws, size_t ws_bytes, void* stream) {
+// The grid search over the rows of one or more weight matrices that share one
+// s (their Delta rows stacked in one buffer, one loss over all of them).
+static int awq_search_pieces(const uint16_t* const* Ws, const int64_t* Ns, int n_mats, int64_t K, const uint16_t* X,
+                             int64_t T, const float* act_mean, const float* alphas, int n_alpha, int group_size,
+                             float* s_out, float* loss_out, int* best_idx, void* ws, size_t ws_bytes, void* stream) {
+  REQUIRE(Ws && Ns && n_mats > 0 && n_mats <= 64, "need 1..64 weight matrices");
+  int64_t N = 0;
+  for (int p = 0; p < n_mats; ++p) {
+    if (int e = check_shape(Ns[p], K)) return e;
+    REQUIRE(Ws[p], "weight matrix %d is NULL", p);
+    REQUIRE(aligned16(Ws[p]), "weight matrix %d must be 16-byte aligned", p);
+    N += Ns[p];
+  }
   if (int e = check_shape(N, K)) return e;
   if (int e = check_group(group_size, K)) return e;
-  REQUIRE_PTR(W);
   if (X) {
     REQUIRE_PTR(X);
     REQUIRE(T > 0, "empty calibration set: X given with T=%lld tokens", (long long)T);
@@ -752,16 +761,23 @@ int awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X,
                              wq::kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B))
       return e;
   }
-  const dim3 dgrid(unsigned((K / 8 + wq::kQuantThreads - 1) / wq::kQuantThreads), unsigned(N));
+  const unsigned gx = unsigned((K / 8 + wq::kQuantThreads - 1) / wq::kQuantThreads);
   for (int i = 0; i < n_alpha; ++i) {
     wq::awq_scale_kernel<<<unsigned((K + 255) / 256), 256, 0, st>>>(a, alphas + i, K, s);
     if (int e = launched("awq_scale launch")) return e;
     double* part_i = partials + int64_t(i) * L.P;
-    if (group_size == 64)
-      wq::awq_delta_kernel<64><<<dgrid, wq::kQuantThreads, 0, st>>>(W, s, N, K, D, a, part_i);
-    else
-      wq::awq_delta_kernel<128><<<dgrid, wq::kQuantThreads, 0, st>>>(W, s, N, K, D, a, part_i);
-    if (int e = launched("awq_delta launch")) return e;
+    int64_t row = 0;  // first stacked row of matrix p
+    for (int p = 0; p < n_mats; ++p) {
+      const dim3 dgrid(gx, unsigned(Ns[p]));
+      uint16_t* Dp = D ? D + row * 2 * K : nullptr;
+      double* pp = D ? part_i : part_i + row * gx;  // proxy partials: one per (row, CTA column)
+      if (group_size == 64)
+        wq::awq_delta_kernel<64><<<dgrid, wq::kQuantThreads, 0, st>>>(Ws[p], s, Ns[p], K, Dp, a, pp);
+      else
+        wq::awq_delta_kernel<128><<<dgrid, wq::kQuantThreads, 0, st>>>(Ws[p], s, Ns[p], K, Dp, a, pp);
+      if (int e = launched("awq_delta launch")) return e;
+      row += Ns[p];
+    }
     if (X) {
       g.sq_partials = part_i;
       const int e = (L.bn == 256) ? launch_gemm_prepared<wq::GEMM_BF16_SQ, 256>(g, st)
@@ -771,6 +787,21 @@ int awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X,
   }
   wq::awq_finalize_kernel<<<1, 256, 0, st>>>(partials, L.P, n_alpha, a, alphas, K, loss_out, best_idx, s_out);
   return launched("awq_finalize launch");
+}
+
+int awq_search_scale(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X, int64_t T, const float* act_mean,
+                     const float* alphas, int n_alpha, int group_size, float* s_out, float* loss_out, int* best_idx,
+                     void* ws, size_t ws_bytes, void* stream) {
+  REQUIRE_PTR(W);
+  return awq_search_pieces(&W, &N, 1, K, X, T, act_mean, alphas, n_alpha, group_size, s_out, loss_out, best_idx, ws,
+                           ws_bytes, stream);
+}
+
+int awq_search_scale_shared(const uint16_t* const* Ws, const int64_t* Ns, int n_mats, int64_t K, const uint16_t* X,
+                            int64_t T, const float* act_mean, const float* alphas, int n_alpha, int group_size,
+                            float* s_out, float* loss_out, int* best_idx, void* ws, size_t ws_bytes, void* stream) {
+  return awq_search_pieces(Ws, Ns, n_mats, K, X, T, act_mean, alphas, n_alpha, group_size, s_out, loss_out, best_idx,
+                           ws, ws_bytes, stream);
 }
 
 int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* qweight,
