@@ -375,6 +375,9 @@ def run_ours(args):
         out["awq_search"] = {"workload": "7 projections, 512 Student-t calibration tokens, 20 alphas, G=64; "
                                          "shared_s: one s for q/k/v and one for gate/up (stacked rows)",
                              "results": awq_measure(wq, synth, torch, dev, peaks)}
+        out["gptq"] = {"workload": "7 projections, 512 Student-t calibration tokens, INT4 G=128 asymmetric, "
+                                   "columns in order",
+                       "results": gptq_measure(wq, synth, torch, dev)}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
     if pg:
@@ -522,6 +525,44 @@ def awq_measure(wq, synth, torch, dev, peaks, T=512):
             "loss_gemm_TFLOP/s": round(tot_flop / tot_s / 1e12, 1),
             "frac_of_bf16_sustained": round(tot_flop / tot_s / 1e12 / peaks["bf16_sustained"], 4),
             "shared_s": shared}
+
+
+def gptq_measure(wq, synth, torch, dev, T=512, G=128):
+    """GPTQ INT4 of the 7 projections (G = 128, asymmetric, T calibration tokens).
+    The inverse-Hessian factor is prepared with PyTorch outside the timed region
+    (its time is reported apart); the timed region is the library's GPTQ kernel.
+    Work: N * K^2 / 2 fused multiply-adds of the error feedback per projection,
+    against the fp32 CUDA-core peak (148 SMs x 128 lanes x 2 flop x max SM clock)."""
+    import time
+    props = torch.cuda.get_device_properties(dev)
+    clock_ghz = 1.965  # max SM clock of this part
+    peak = props.multi_processor_count * 128 * 2 * clock_ghz / 1e3  # TFLOP/s
+    per, tot_s, tot_flop, prep_s = {}, 0.0, 0.0, 0.0
+    for name, K, N in synth.PROJECTIONS:
+        W = synth.weight(N, K, seed=synth.layer_seed(6, K + N), device=dev)
+        X = synth.activations_student_t(T, K, seed=synth.layer_seed(6, K), device=dev)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        U = wq.gptq_hessian_factor(X)
+        torch.cuda.synchronize()
+        prep_s += time.perf_counter() - t0
+        wq.wq_gptq_int4(W, U, G, 1)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        wq.wq_gptq_int4(W, U, G, 1)
+        b.record()
+        torch.cuda.synchronize()
+        sec = a.elapsed_time(b) * 1e-3
+        flop = float(N) * K * K  # 2 flop per fused multiply-add, K^2 / 2 of them per row
+        per[name] = {"ms": round(sec * 1e3, 3), "TFLOP/s": round(flop / sec / 1e12, 2)}
+        tot_s += sec
+        tot_flop += flop
+        del U, W, X
+    return {"ms_per_projection": per, "ms_total": round(tot_s * 1e3, 3),
+            "TFLOP/s": round(tot_flop / tot_s / 1e12, 2), "peak_fp32_TFLOP/s": round(peak, 1),
+            "frac_of_fp32_peak": round(tot_flop / tot_s / 1e12 / peak, 4), "bound": "alu",
+            "input_preparation_s": round(prep_s, 3)}
 
 
 # ---------------------------------------------------------------- oracle arm

@@ -126,6 +126,29 @@ int wq_quantize_int4(const uint16_t* W, int64_t N, int64_t K, int bits, int grou
 int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scale_s,
                       uint8_t* codes, uint8_t* bscale, float* global_scale, void* stream);
 
+/* wq_gptq_int4 -- GPTQ INT4 quantize-and-pack with second-order error
+ * feedback ("quantization primer" section 6 "GPTQ": quantize a weight,
+ * estimate its error with second-order information, adjust the weights not
+ * yet quantized, continue; ms-swift page: Hessian from calibration samples,
+ * group size 128, no activation reordering).
+ *   W        bf16 [N, K], 16-byte aligned
+ *   U        fp32 [K, K] row-major, device: the upper Cholesky factor of the
+ *            damped inverse Hessian, U^T U = (2 X^T X + lambda I)^-1 over the
+ *            caller's calibration tokens X (only the upper triangle is read)
+ *   group_size, zero_point, qweight, scales, zeros: as wq_quantize_int4, and
+ *            the same packed format (so every linear entry point takes it)
+ * Per row, columns k = 0..K-1 in order: at a group's first column its scale
+ * and zero point follow wq_quantize_int4's rule applied to the group's
+ * weights as they stand; q_k as wq_quantize_int4;
+ * e_k = (w_k - (q_k - z) * scale) / U[k][k]; then w_j = fmaf(-e_k, U[k][j], w_j)
+ * for all j > k.  All in fp32, one rounding per operation, every w_j adjusted
+ * in increasing k: the codes are bit-for-bit deterministic.  Returns
+ * WQ_ERR_UNSUPPORTED if one row of K fp32 weights plus a G x G tile of U does
+ * not fit the GPU's shared memory (K up to ~40000). */
+int wq_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int group_size,
+                 int zero_point, uint32_t* qweight, uint16_t* scales, uint32_t* zeros,
+                 void* stream);
+
 /* awq_search_scale -- AWQ grid search of the per-input-channel scale
  * ("Lance-Quant" section "量化应用": grid-search AWQ scale equalization;
  * "quantization primer" section 7: scale salient channels by activation

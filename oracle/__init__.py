@@ -75,6 +75,8 @@ def _L():
         lib.oracle_awq_delta.argtypes = [P, I64, I64, P, I, P]
         lib.oracle_awq_search.restype = I
         lib.oracle_awq_search.argtypes = [P, I64, I64, P, I64, P, P, I, I, P, P, P]
+        lib.oracle_gptq_int4.restype = I
+        lib.oracle_gptq_int4.argtypes = [P, I64, I64, P, I, I, P, P, P, P]
         lib.oracle_num_threads.restype = I
         lib.oracle_num_threads.argtypes = []
         _lib = lib
@@ -256,3 +258,44 @@ def awq_search(W, group_size: int, alphas, X=None, act_mean=None):
     if rc != 0:
         raise ValueError("oracle_awq_search: invalid arguments")
     return s, losses, best.value
+
+
+def gptq_hessian_factor(X, damp: float = 0.01) -> np.ndarray:
+    """U (fp32 [K, K], upper triangular) with U^T U = (H + lambda I)^-1, where
+    H = 2 X^T X over the calibration tokens X [T, K] and lambda = damp times the
+    mean of diag(H) ("quantization primer" section 6 and the ms-swift page: the
+    second-order information of GPTQ comes from 128-512 calibration samples;
+    the damping is a reading, the pages are silent).  fp64 throughout, numpy's
+    inverse and Cholesky factorisation as library steps, rounded to fp32 once."""
+    x = activations_f64(X)
+    H = 2.0 * (x.T @ x)
+    K = H.shape[0]
+    H[np.diag_indices(K)] += damp * np.mean(np.diag(H))
+    Hinv = np.linalg.inv(H)
+    Hinv = 0.5 * (Hinv + Hinv.T)
+    return np.ascontiguousarray(np.linalg.cholesky(Hinv).T.astype(np.float32))
+
+
+def gptq_int4(W, U, group_size: int, zero_point: int = 1, want_err: bool = False) -> dict:
+    """GPTQ INT4 pack of W [N, K] with the inverse-Hessian factor U (fp32 [K, K]):
+    columns in order, group scale/zero from the weights as they stand at the
+    group's first column, error e_k = (w_k - deq(q_k)) / U[k][k], later columns
+    w_j -= e_k U[k][j] in fp32.  Returns the pack (and e [N, K] fp32)."""
+    w = as_bits16(W)
+    N, K = w.shape
+    u = np.ascontiguousarray(U, dtype=np.float32)
+    if u.shape != (K, K):
+        raise ValueError("U must be [K, K]")
+    ng = K // group_size
+    out = {"qweight": np.zeros((N, K // 8), dtype=np.uint32),
+           "scales": np.zeros((N, ng), dtype=np.uint16),
+           "zeros": np.zeros((N, (ng + 7) // 8), dtype=np.uint32) if zero_point else None}
+    err = np.zeros((N, K), dtype=np.float32) if want_err else None
+    rc = _L().oracle_gptq_int4(_ptr(w), N, K, _ptr(u), group_size, zero_point, _ptr(out["qweight"]),
+                               _ptr(out["scales"]), _ptr(out["zeros"]), _ptr(err))
+    if rc != 0:
+        raise ValueError("oracle_gptq_int4: invalid arguments")
+    out.update(N=N, K=K, group_size=group_size, zero_point=zero_point)
+    if want_err:
+        out["err"] = err
+    return out

@@ -21,6 +21,8 @@
  *       has no calibration activations (section "校准阶段").
  *  [P2] "OmniQuant" tutorial (cyqw.cn), section 2.1 (scale and zero point)
  *       and section 2.2.2 (equivalence transform Y = (X s)(W / s)).
+ *  [P4] section 6 "GPTQ": quantize, estimate the error with second-order
+ *       information, adjust the remaining weights, continue.
  *  Where the pages are silent the readings used here are listed next to the
  *  code that takes them (min-max range, 1e-5 scale floor, fp16 scale,
  *  LSB-first nibble order, NVFP4 per-tensor scale amax/(6*448), E2M1 ties to
@@ -417,6 +419,80 @@ int oracle_awq_search(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X
   *best_out = best;
   free(a); free(s); free(delta); free(xd); free(y);
   return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* GPTQ ([P4] section 6 "GPTQ")                                          */
+/* ------------------------------------------------------------------ */
+
+/* GPTQ INT4 quantize-and-pack.  The page gives the loop only: quantize a
+ * weight, estimate its error with approximate second-order information,
+ * adjust the weights not yet quantized, continue; 4-bit weights, calibration
+ * data, group size 128 and no activation reordering in its example.
+ * Readings taken here:
+ *  - the second-order information is the upper Cholesky factor U of the
+ *    damped inverse Hessian of the calibration activations (U^T U =
+ *    (2 X^T X + lambda I)^-1), given by the caller in fp32;
+ *  - columns are quantized in order k = 0..K-1, every row on its own;
+ *  - a group's scale and zero point come from the plain quantizer's min-max
+ *    rule applied to the group's weights as they stand when its first column
+ *    is reached (after the adjustments from earlier columns);
+ *  - the error of column k is e_k = (w_k - dequant(q_k)) / U[k][k] and the
+ *    adjustment of every later column j is w_j = fmaf(-e_k, U[k][j], w_j),
+ *    in fp32 (the precision the GPU kernel takes the same decisions in), one
+ *    rounding per operation, k in increasing order.
+ * In exact arithmetic this gives W - dequant(Q) = E U row by row, which the
+ * tests check.  err (optional, fp32 [N, K]) receives the e_k. */
+int oracle_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int group_size, int zero_point,
+                     uint32_t* qweight, uint16_t* scales, uint32_t* zeros, float* err) {
+  if (N <= 0 || K <= 0 || group_size <= 0 || K % group_size || K % 8 || !U) return ORACLE_ERR_ARG;
+  if (zero_point && !zeros) return ORACLE_ERR_ARG;
+  const int64_t G = group_size, ng = K / G, nzw = (ng + 7) / 8;
+  memset(qweight, 0, (size_t)(N * (K / 8)) * sizeof(uint32_t));
+  if (zero_point) memset(zeros, 0, (size_t)(N * nzw) * sizeof(uint32_t));
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t n = 0; n < N; ++n) {
+    float* w = (float*)malloc((size_t)K * sizeof(float));
+    if (!w) {
+#pragma omp atomic write
+      bad = 1;
+      continue;
+    }
+    for (int64_t k = 0; k < K; ++k) w[k] = bf16_to_f32(W[n * K + k]);
+    float sc = 1.0f, z = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+      if (k % G == 0) {  /* the group's scale and zero point from its current weights */
+        const int64_t g = k / G;
+        float mn = INFINITY, mx = -INFINITY, amax = 0.0f;
+        for (int64_t i = k; i < k + G; ++i) {
+          if (w[i] < mn) mn = w[i];
+          if (w[i] > mx) mx = w[i];
+          if (fabsf(w[i]) > amax) amax = fabsf(w[i]);
+        }
+        if (zero_point) {
+          scales[n * ng + g] = group_scale(mx - mn, 15.0f, &sc);
+          z = clampf(rintf(-mn / sc), 0.0f, 15.0f);
+          zeros[n * nzw + g / 8] |= (uint32_t)z << (4 * (g % 8));
+        } else {
+          scales[n * ng + g] = group_scale(amax, 7.0f, &sc);
+          z = 8.0f;
+        }
+      }
+      /* quantize the weight */
+      const float q = zero_point ? clampf(rintf(w[k] / sc) + z, 0.0f, 15.0f)
+                                 : clampf(rintf(w[k] / sc), -7.0f, 7.0f) + 8.0f;
+      qweight[n * (K / 8) + k / 8] |= (uint32_t)q << (4 * (k % 8));
+      /* estimate its error, scaled by the second-order information */
+      const float deq = (q - z) * sc; /* exact: |q - z| <= 15, sc has 11 significant bits */
+      const float e = (w[k] - deq) / U[k * K + k];
+      if (err) err[n * K + k] = e;
+      /* adjust the weights not yet quantized */
+      for (int64_t j = k + 1; j < K; ++j) w[j] = fmaf(-e, U[k * K + j], w[j]);
+    }
+    free(w);
+  }
+  return bad ? ORACLE_ERR_ARG : ORACLE_OK;
 }
 
 int oracle_num_threads(void) {

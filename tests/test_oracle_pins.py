@@ -415,3 +415,59 @@ def test_awq_shared_scale_is_the_search_over_stacked_rows():
         s, shared, best = oracle.awq_search(torch.cat(Ws), G, ALPHAS, **kw)
         np.testing.assert_allclose(shared, parts, rtol=1e-12)
         assert best == int(np.argmin(parts))
+
+
+# ---------------------------------------------------------------- GPTQ
+def _spd_factor(K, seed, corr=0.9):
+    # calibration tokens with strongly correlated channels (so that the second-order
+    # adjustment matters), and the inverse-Hessian factor from them
+    rng = np.random.default_rng(seed)
+    base = rng.standard_normal((256, K // 4))
+    x = np.repeat(base, 4, axis=1) * corr + rng.standard_normal((256, K)) * (1 - corr)
+    X = _bf16(x.astype(np.float32))
+    return X, oracle.gptq_hessian_factor(X)
+
+
+@pytest.mark.parametrize("zp", [1, 0])
+def test_gptq_identity_factor_is_plain_rtn(zp):
+    # U = I: no second-order coupling, nothing to adjust -> the plain min-max quantizer
+    # ("quantization primer" section 6 reduces to sections 2-3), and e = w - deq(q)
+    N, K, G = 16, 256, 64
+    W = synth.weight(N, K, seed=60, outlier_frac=0.02)
+    g = oracle.gptq_int4(W, np.eye(K, dtype=np.float32), G, zp, want_err=True)
+    r = oracle.quantize_int4(W, G, zp)
+    for key in ("qweight", "scales", "zeros"):
+        if r[key] is not None:
+            np.testing.assert_array_equal(g[key], r[key])
+    np.testing.assert_array_equal(g["err"], (W.float().numpy() - oracle.dequant_int4(r)).astype(np.float32))
+
+
+@pytest.mark.parametrize("G", [64, 128])
+def test_gptq_error_identity(G):
+    # The adjustments accumulate so that w - deq(q) = e U for every row (U upper
+    # triangular): column j carries e_k U[k][j] from every k < j plus its own
+    # e_j U[j][j].  A dropped, mis-signed or transposed term breaks it.
+    N, K = 12, 256
+    W = synth.weight(N, K, seed=61, outlier_frac=0.02)
+    _, U = _spd_factor(K, 61)
+    g = oracle.gptq_int4(W, U, G, want_err=True)
+    lhs = W.double().numpy() - oracle.dequant_int4(g)
+    rhs = g["err"].astype(np.float64) @ np.triu(U).astype(np.float64)
+    np.testing.assert_allclose(lhs, rhs, rtol=0, atol=2e-5 * np.abs(W.double().numpy()).max())
+
+
+def test_gptq_factor_and_loss():
+    # U^T U is the damped inverse Hessian; GPTQ's output error under H, |X (W - Q)^T|^2,
+    # beats plain rounding on correlated calibration data (the point of the method)
+    N, K, G = 24, 256, 64
+    W = synth.weight(N, K, seed=62, outlier_frac=0.02)
+    X, U = _spd_factor(K, 62)
+    x = X.double().numpy()
+    H = 2 * x.T @ x
+    H[np.diag_indices(K)] += 0.01 * np.mean(np.diag(H))
+    np.testing.assert_allclose(U.astype(np.float64).T @ U.astype(np.float64), np.linalg.inv(H),
+                               rtol=0, atol=1e-6 * np.abs(np.linalg.inv(H)).max())
+    assert np.all(np.tril(U, -1) == 0)
+    w = W.double().numpy()
+    loss = lambda q: float(np.sum((x @ (w - oracle.dequant_int4(q)).T) ** 2))
+    assert loss(oracle.gptq_int4(W, U, G)) < 0.8 * loss(oracle.quantize_int4(W, G))

@@ -8,7 +8,7 @@ library's CUDA kernels.  There is no CPU fallback: if the library cannot be
 loaded every call raises.
 
 Functions carry the C names:
-    wq_quantize_int4, wq_quantize_nvfp4, awq_search_scale, awq_search_scale_shared,
+    wq_quantize_int4, wq_gptq_int4, wq_quantize_nvfp4, awq_search_scale, awq_search_scale_shared,
     wq_linear_int4, wq_linear_nvfp4, wq_linear_group, wq_device_error
 """
 from __future__ import annotations
@@ -36,6 +36,7 @@ SIGNATURES = {
     "wq_linear_workspace_size": (_I, [_I64, _I64, _I64, _I, _I, _PSZ]),
     "awq_search_workspace_size": (_I, [_I64, _I64, _I64, _I, _I, _PSZ]),
     "wq_quantize_int4": (_I, [_P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "wq_gptq_int4": (_I, [_P, _I64, _I64, _P, _I, _I, _P, _P, _P, _P]),
     "wq_quantize_nvfp4": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "awq_search_scale": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "awq_search_scale_shared": (_I, [_P, _P, _I, _I64, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P]),
@@ -173,6 +174,40 @@ def wq_quantize_int4(W: torch.Tensor, group_size: int = 64, zero_point: int = 1,
     _check(lib.wq_quantize_int4(_ptr(W), N, K, bits, group_size, zero_point, _ptr(s), _ptr(qweight),
                                 _ptr(scales), _ptr(zeros), _stream()), "wq_quantize_int4")
     return PackedInt4(qweight, scales, zeros, N, K, group_size, zero_point)
+
+
+def wq_gptq_int4(W: torch.Tensor, U: torch.Tensor, group_size: int = 128, zero_point: int = 1) -> PackedInt4:
+    """GPTQ INT4 pack of W with the inverse-Hessian factor U (fp32 [K, K] upper
+    Cholesky factor of the damped inverse Hessian; see gptq_hessian_factor).
+    Same packed format as wq_quantize_int4."""
+    if isinstance(W, (PackedInt4, PackedNVFP4)):
+        raise ValueError("the layer is already quantized")
+    _dev(W, "W", torch.bfloat16)
+    N, K = W.shape
+    _dev(U, "U", torch.float32)
+    if tuple(U.shape) != (K, K):
+        raise ValueError(f"U must be [{K}, {K}]")
+    lib = load()
+    ng = K // group_size if group_size and K % group_size == 0 else 1
+    qweight = torch.empty((N, max(K // 8, 1)), dtype=torch.int32, device=W.device)
+    scales = torch.empty((N, ng), dtype=torch.float16, device=W.device)
+    zeros = torch.empty((N, (ng + 7) // 8), dtype=torch.int32, device=W.device) if zero_point else None
+    _check(lib.wq_gptq_int4(_ptr(W), N, K, _ptr(U), group_size, zero_point, _ptr(qweight), _ptr(scales),
+                            _ptr(zeros), _stream()), "wq_gptq_int4")
+    return PackedInt4(qweight, scales, zeros, N, K, group_size, zero_point)
+
+
+def gptq_hessian_factor(X: torch.Tensor, damp: float = 0.01) -> torch.Tensor:
+    """Input preparation for wq_gptq_int4, outside the library: U (fp32 [K, K],
+    upper) with U^T U = (H + lambda I)^-1, H = 2 X^T X over calibration tokens X
+    [T, K], lambda = damp * mean(diag H).  Runs PyTorch's fp64 linear algebra
+    (matmul, Cholesky, inverse) on X's device; the quantization itself runs in
+    the library's kernel."""
+    x = X.to(torch.float64)
+    H = 2.0 * (x.T @ x)
+    H.diagonal().add_(damp * H.diagonal().mean())
+    Hinv = torch.cholesky_inverse(torch.linalg.cholesky(H))
+    return torch.linalg.cholesky(Hinv, upper=True).to(torch.float32).contiguous()
 
 
 def wq_quantize_nvfp4(W: torch.Tensor, scale_s=None) -> PackedNVFP4:

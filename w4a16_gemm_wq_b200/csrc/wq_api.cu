@@ -17,6 +17,7 @@
 #include "gemm_tcgen05.cuh"
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
+#include "gptq.cuh"
 #include "quant.cuh"
 #include "wq_common.cuh"
 
@@ -697,6 +698,45 @@ int wq_quantize_int4(const uint16_t* W, int64_t N, int64_t K, int bits, int grou
       wq::quantize_int4_kernel<128, false><<<grid, wq::kQuantThreads, 0, st>>>(W, scale_s, N, K, qweight, scales, zeros);
   }
   return launched("quantize_int4 launch");
+}
+
+int wq_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int group_size, int zero_point,
+                 uint32_t* qweight, uint16_t* scales, uint32_t* zeros, void* stream) {
+  if (int e = check_shape(N, K)) return e;
+  if (int e = check_group(group_size, K)) return e;
+  REQUIRE(zero_point == 0 || zero_point == 1, "zero_point must be 0 or 1");
+  REQUIRE_PTR(W);
+  REQUIRE(aligned16(W), "W must be 16-byte aligned");
+  REQUIRE_PTR(U);
+  REQUIRE_PTR(qweight);
+  REQUIRE_PTR(scales);
+  if (zero_point) {
+    REQUIRE_PTR(zeros);
+  } else {
+    REQUIRE(!zeros, "zeros must be NULL for a symmetric (zero_point=0) pack");
+  }
+  int dev = 0, optin = 0, sms = 0;
+  if (int e = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return e;
+  if (int e = cuda_check(cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev), "smem attr"))
+    return e;
+  if (int e = cuda_check(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "SM count")) return e;
+  const int G = group_size;
+  const int64_t fit = (int64_t(optin) - int64_t(G) * G * 4) / (K * 4 + int64_t(G) * 5);
+  const int R = int(std::min<int64_t>({int64_t(wq::kGptqMaxRows), N, fit}));
+  if (R < 1) return fail(WQ_ERR_UNSUPPORTED, "K = %lld is too long for one row in shared memory", (long long)K);
+  wq::GptqArgs a = {W, U, N, K, R, qweight, scales, zeros};
+  const size_t smem = wq::gptq_smem_bytes(R, K, G);
+  const unsigned grid = unsigned(std::min<int64_t>((N + R - 1) / R, sms));
+  cudaStream_t st = as_stream(stream);
+  const auto go = [&](auto kern) -> int {
+    if (int e = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)),
+                           "gptq smem attribute"))
+      return e;
+    kern<<<grid, wq::kGptqThreads, smem, st>>>(a);
+    return launched("gptq_int4 launch");
+  };
+  if (G == 64) return zero_point ? go(wq::gptq_int4_kernel<64, true>) : go(wq::gptq_int4_kernel<64, false>);
+  return zero_point ? go(wq::gptq_int4_kernel<128, true>) : go(wq::gptq_int4_kernel<128, false>);
 }
 
 int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scale_s, uint8_t* codes,
