@@ -185,18 +185,32 @@ __device__ __forceinline__ uint4 dequant_word_int4(uint32_t w, uint32_t zoff2, u
 }
 
 // NVFP4: one packed word (codes of k = 8j..8j+7, low nibble = even k) -> 8 bf16
-// e2m1 * sb, natural order.  The product is formed in f16 (exact: at most 6
-// significant bits, |v| <= 6 * 448) and then rounded to bf16 (exact as well).
-__device__ __forceinline__ uint32_t e2m1x2_scaled_bf16x2(uint32_t byte, uint32_t sb2) {
-  uint32_t h;
-  asm("{ .reg .b8 q; cvt.u8.u32 q, %1; cvt.rn.f16x2.e2m1x2 %0, q; }" : "=r"(h) : "r"(byte));
-  asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(h) : "r"(sb2));
-  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
-  return pack_bf16x2(f.x, f.y);
+// e2m1 * sb, natural order, with integer and bf16 ALU operations only (no
+// conversion instructions): the bf16 bytes of |e2m1| come from two byte
+// lookups (prmt over an 8-entry table: magnitude index = the code's low 3
+// bits), the bf16 block scale sb2 = {sb, sb} multiplies them (exact: at most
+// 6 significant bits, |v| <= 6 * 448), and each code's sign bit is OR-ed into
+// its product.
+__device__ __forceinline__ uint32_t lop3_or_and(uint32_t a, uint32_t b, uint32_t c) {  // a | (b & c)
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xF8;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 __device__ __forceinline__ uint4 dequant_word_nvfp4(uint32_t w, uint32_t sb2) {
-  return make_uint4(e2m1x2_scaled_bf16x2(w & 0xFF, sb2), e2m1x2_scaled_bf16x2((w >> 8) & 0xFF, sb2),
-                    e2m1x2_scaled_bf16x2((w >> 16) & 0xFF, sb2), e2m1x2_scaled_bf16x2(w >> 24, sb2));
+  // bf16 of 0, 0.5, 1, 1.5 | 2, 3, 4, 6: low bytes and high bytes, table index = byte index
+  constexpr uint32_t kLoA = 0xC0800000u, kLoB = 0xC0804000u, kHiA = 0x3F3F3F00u, kHiB = 0x40404040u;
+  const uint32_t s0 = w & 0x7777u, s1 = (w >> 16) & 0x7777u;  // magnitude indices of codes 0-3, 4-7
+  const uint32_t l0 = prmt_b32(kLoA, kLoB, s0), h0 = prmt_b32(kHiA, kHiB, s0);
+  const uint32_t l1 = prmt_b32(kLoA, kLoB, s1), h1 = prmt_b32(kHiA, kHiB, s1);
+  // {code 2i, code 2i+1} as bf16x2 magnitudes, times the block scale
+  const uint32_t m0 = bf16x2_mul(prmt_b32(l0, h0, 0x5140), sb2), m1 = bf16x2_mul(prmt_b32(l0, h0, 0x7362), sb2);
+  const uint32_t m2 = bf16x2_mul(prmt_b32(l1, h1, 0x5140), sb2), m3 = bf16x2_mul(prmt_b32(l1, h1, 0x7362), sb2);
+  // sign of code 2i (bit 8i+3 of w = bit 7 of byte i of w << 4) -> bit 15, of code 2i+1 (bit 7 of byte i of w) -> bit 31
+  const uint32_t t = w << 4;
+  return make_uint4(lop3_or_and(m0, prmt_b32(t, w, 0x4000), 0x80008000u),
+                    lop3_or_and(m1, prmt_b32(t, w, 0x5010), 0x80008000u),
+                    lop3_or_and(m2, prmt_b32(t, w, 0x6020), 0x80008000u),
+                    lop3_or_and(m3, prmt_b32(t, w, 0x7030), 0x80008000u));
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
@@ -332,8 +346,12 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
         const int nb = a.K >> 4;
         const uint8_t* bs = a.bscale + int64_t(n) * nb + kb * 4;
         const int rem = nb - kb * 4;  // K % 64 == 32 leaves two blocks in the last k-block
-        raw_a = 0;
-        for (int q = 0; q < 4 && q < rem; ++q) raw_a |= uint32_t(__ldg(bs + q)) << (8 * q);
+        if (rem >= 4 && (reinterpret_cast<uintptr_t>(bs) & 3) == 0) {
+          raw_a = __ldg(reinterpret_cast<const uint32_t*>(bs));  // the k-block's 4 scales in one load
+        } else {
+          raw_a = 0;
+          for (int q = 0; q < 4 && q < rem; ++q) raw_a |= uint32_t(__ldg(bs + q)) << (8 * q);
+        }
       }
     };
     uint32_t meta_a, meta_b;
@@ -343,7 +361,7 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
       const uint32_t cur_a = meta_a, cur_b = meta_b;
       fetch_meta(kb + 1, meta_a, meta_b);
       uint32_t sc2 = 0, zoff2 = 0;
-      uint32_t sbv[4] = {0, 0, 0, 0};  // NVFP4: the k-block's 4 E4M3 block scales as f16x2 {sb, sb}
+      uint32_t sbv[4] = {0, 0, 0, 0};  // NVFP4: the k-block's 4 E4M3 block scales as bf16x2 {sb, sb}
       if (FMT == GEMM_INT4) {
         const int g = (kb * kGemmBK) >> a.log2g;
         const float sc = __half2float(__ushort_as_half(uint16_t(cur_a)));
@@ -353,12 +371,13 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
         zoff2 = zb | (zb << 16);
       } else {
 #pragma unroll
-        for (int q = 0; q < 4; q += 2) {  // two E4M3 bytes -> f16x2 (exact), then replicate each
+        for (int q = 0; q < 4; q += 2) {  // two E4M3 bytes -> f16x2 -> fp32 -> bf16 (all exact), then replicate each
           uint32_t h2;
           asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }"
               : "=r"(h2) : "r"((cur_a >> (8 * q)) & 0x7F7Fu));
-          sbv[q] = __byte_perm(h2, 0, 0x1010);
-          sbv[q + 1] = __byte_perm(h2, 0, 0x3232);
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+          sbv[q] = pack_bf16x2(f.x, f.x);
+          sbv[q + 1] = pack_bf16x2(f.y, f.y);
         }
       }
       if (!mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag)) { ok = false; break; }
