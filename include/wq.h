@@ -81,9 +81,13 @@ int wq_int4_sizes(int64_t N, int64_t K, int group_size, size_t* qweight_bytes,
                   size_t* scales_bytes, size_t* zeros_bytes);
 int wq_nvfp4_sizes(int64_t N, int64_t K, size_t* codes_bytes, size_t* bscale_bytes);
 
-/* Scratch bytes wq_linear_int4 / wq_linear_nvfp4 need for an [M, K] x [N, K]
- * problem (format WQ_FMT_*, act_fp4 as in wq_linear_nvfp4).  0 means the call
- * needs no workspace and accepts ws = NULL (every W4A16 call; W4A4 needs one). */
+/* Scratch bytes wq_linear_int4 / wq_linear_nvfp4 use for an [M, K] x [N, K]
+ * problem (format WQ_FMT_*, act_fp4 as in wq_linear_nvfp4).  W4A4 requires a
+ * workspace of this size.  W4A16 never requires one: a non-zero size means a
+ * prefill GEMM with few output tiles (under half the SMs) that, given a
+ * workspace of at least this size, splits K over several CTAs per tile (fp32
+ * partials summed in split order by the last CTA of each tile, so the result
+ * does not depend on timing); with ws = NULL or a smaller one it runs unsplit. */
 int wq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int format, int act_fp4,
                              size_t* bytes);
 
@@ -200,8 +204,9 @@ int awq_search_scale_shared(const uint16_t* const* Ws, const int64_t* Ns, int n_
  *   act_inv_s fp32 [K] or NULL: multiplies column k of X (the 1/s of an AWQ
  *            scale that could not be folded into a preceding norm)
  *   Y        bf16 [M, N]
- *   ws, ws_bytes: scratch of at least wq_linear_workspace_size bytes (may be
- *            NULL when that size is 0)
+ *   ws, ws_bytes: optional scratch (NULL allowed): with at least
+ *            wq_linear_workspace_size bytes, a prefill GEMM with few output
+ *            tiles splits K over several CTAs per tile
  * M <= 16 runs the split-K CUDA-core decode GEMV (one launch, lowest
  * latency for a single projection); larger M runs the tensor-core GEMM.
  * wq_linear_group runs decode projections on the tensor-core decode GEMV. */

@@ -112,3 +112,30 @@ def test_two_accumulator_tiles_ragged(lib, M, N, fmt):
     rows = np.array(sorted(set(range(120, 264, 3)) | set(range(2040, 2300, 7)) | {M - 1}))
     ref = oracle.linear(X[rows].cpu(), _deq(p), None if inv_s is None else inv_s.cpu().numpy())
     assert_linear_close(Y[rows], ref, what=f"{fmt} M={M} N={N}")
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+@pytest.mark.parametrize("M,N,K", [(512, 256, 11008), (2048, 256, 4096), (512, 2048, 11008), (300, 200, 3072)])
+def test_split_k_few_tiles(lib, fmt, M, N, K):
+    # few output tiles: K split over several CTAs per tile through the workspace
+    # (fp32 partials, the last CTA of a tile sums them in split order): sampled rows
+    # against the oracle, bit-identical on a second run with the same workspace (the
+    # counters start as garbage and must come back to 0), and close to the unsplit run
+    W = synth.weight(N, K, seed=M + N + K, device="cuda")
+    X = synth.activations(M, K, seed=K, device="cuda")
+    p = lib.wq_quantize_int4(W, 64, 1) if fmt == "int4" else lib.wq_quantize_nvfp4(W)
+    call = lib.wq_linear_int4 if fmt == "int4" else lib.wq_linear_nvfp4
+    fmt_id = lib.WQ_FMT_INT4 if fmt == "int4" else lib.WQ_FMT_NVFP4
+    need = lib.linear_workspace_size(M, N, K, fmt_id)
+    assert need > 0, "these shapes take the split"
+    ws = torch.full((need,), 0xAB, dtype=torch.uint8, device="cuda")
+    y1 = call(X, p, ws=ws).clone()
+    y2 = call(X, p, ws=ws).clone()
+    y0 = call(X, p, ws=torch.empty(16, dtype=torch.uint8, device="cuda"))  # too small: unsplit
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16)), "split sums must not depend on timing"
+    rows = _sampled_rows(M)
+    ref = oracle.linear(X[rows].cpu(), _deq(p))
+    assert_linear_close(y1[rows], ref, what=f"split-K {fmt} {M}x{N}x{K}")
+    assert_linear_close(y0[rows], ref, what=f"unsplit {fmt} {M}x{N}x{K}")
+    assert lib.wq_device_error() == 0

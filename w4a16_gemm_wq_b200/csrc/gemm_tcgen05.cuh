@@ -68,6 +68,9 @@ struct GemmArgs {
   const float* inv_s;       // fp32 [K] or null
   uint16_t* Y;              // bf16 [M, N]
   double* sq_partials;      // FMT_BF16_SQ: one partial sum of squares per epilogue warp
+  float* part;              // split-K: fp32 partial tiles [tiles][splitk][BMT * BN]
+  unsigned* ctr;            // split-K: arrivals per tile (0 before and after a launch)
+  int splitk;               // CTAs per output tile along K (gridDim.z); 1 = no split
   int M, N, K;              // K: reduction length (for FMT_BF16_SQ the length of B's rows)
   int a_kblocks;            // A k-block index wraps modulo this (FMT_BF16_SQ reuses X twice)
   int log2g;
@@ -245,10 +248,15 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
   uint64_t* accum = bars + 3 * STAGES;   // accumulator complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* split_last = reinterpret_cast<volatile int*>(tmem_slot + 2);  // split-K: this CTA sums the tile
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * BMT, n0 = blockIdx.x * BN;
-  const int nkb = (a.K + kGemmBK - 1) / kGemmBK;
+  const int nkb_all = (a.K + kGemmBK - 1) / kGemmBK;
+  // split-K: this CTA's k-blocks [kbeg, kbeg + nkb)
+  const int splits = a.splitk > 1 ? a.splitk : 1;
+  const int kbeg = int((int64_t(nkb_all) * blockIdx.z) / splits);
+  const int nkb = int((int64_t(nkb_all) * (blockIdx.z + 1)) / splits) - kbeg;
   constexpr int DEQ_WARP0 = 4;
   constexpr int DEQ_WARPS = S::DEQ_THREADS / 32;
 
@@ -281,8 +289,8 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
     if (lane == 0) {
       asm volatile("griddepcontrol.wait;" ::: "memory");
       int issued = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % STAGES, r = kb / STAGES;
+      for (int i = 0; i < nkb; ++i) {
+        const int kb = kbeg + i, s = i % STAGES, r = i / STAGES;
         if (r > 0 && !mbar_wait(&empty[s], (r - 1) & 1, ERR_TIMEOUT_PIPE, abort_flag)) break;
         if (FMT == GEMM_BF16_SQ) {
           mbar_arrive_expect_tx(&full[s], S::A_BYTES + S::B_BYTES);
@@ -306,8 +314,8 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC = idesc_bf16_f32(kGemmBM, BN);
       bool ok = true;
-      for (int kb = 0; kb < nkb && ok; ++kb) {
-        const int s = kb % STAGES, r = kb / STAGES;
+      for (int i = 0; i < nkb && ok; ++i) {
+        const int s = i % STAGES, r = i / STAGES;
         ok = mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag) &&
              (FMT == GEMM_BF16_SQ || mbar_wait(&bready[s], r & 1, ERR_TIMEOUT_PIPE, abort_flag));
         if (!ok) break;
@@ -316,10 +324,10 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
         const uint64_t bd = desc_kmajor_sw128(b_addr(s));
 #pragma unroll
         for (int kk = 0; kk < kGemmBK / 16; ++kk) {  // +32 bytes per K=16 step inside the swizzle atom
-          umma_bf16(tmem_acc, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), IDESC, (kb | kk) != 0);
+          umma_bf16(tmem_acc, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), IDESC, (i | kk) != 0);
           if (S::NACC == 2)  // rows 128-255 of the X tile start 16 KB (16 atoms) further
             umma_bf16(tmem_acc + BN, desc_kmajor_sw128(a_addr(s) + 16384) + uint64_t(2 * kk),
-                      bd + uint64_t(2 * kk), IDESC, (kb | kk) != 0);
+                      bd + uint64_t(2 * kk), IDESC, (i | kk) != 0);
         }
         umma_commit(&empty[s]);
       }
@@ -337,7 +345,7 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
     auto fetch_meta = [&](int kb, uint32_t& raw_a, uint32_t& raw_b) {
       raw_a = 0;
       raw_b = 0x88888888u;
-      if (kb >= nkb) return;
+      if (kb >= kbeg + nkb) return;
       if (FMT == GEMM_INT4) {
         const int g = (kb * kGemmBK) >> a.log2g;
         raw_a = __ldg(a.scales + int64_t(n) * ng + g);
@@ -355,9 +363,9 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
       }
     };
     uint32_t meta_a, meta_b;
-    fetch_meta(0, meta_a, meta_b);
-    for (int kb = 0; kb < (FMT == GEMM_BF16_SQ ? 0 : nkb); ++kb) {
-      const int s = kb % STAGES, r = kb / STAGES;
+    fetch_meta(kbeg, meta_a, meta_b);
+    for (int i = 0; i < (FMT == GEMM_BF16_SQ ? 0 : nkb); ++i) {
+      const int kb = kbeg + i, s = i % STAGES, r = i / STAGES;
       const uint32_t cur_a = meta_a, cur_b = meta_b;
       fetch_meta(kb + 1, meta_a, meta_b);
       uint32_t sc2 = 0, zoff2 = 0;
@@ -408,13 +416,84 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
     // ---------------------------------------------------------- epilogue
     bool go = ok && mbar_wait(accum, 0, ERR_TIMEOUT_MMA, abort_flag);
     go = __all_sync(0xffffffffu, go);  // tcgen05.ld below is warp-collective
-    if (go) {
-      tc_fence_after();
-      const int quarter = warp & 3;                      // TMEM lanes 32*quarter .. +31
-      constexpr int WPQ = DEQ_WARPS / 4;                 // epilogue warps per lane quarter
-      const int wi = (warp - DEQ_WARP0) >> 2;            // this warp's index among them
+    const int quarter = warp & 3;                      // TMEM lanes 32*quarter .. +31
+    constexpr int WPQ = DEQ_WARPS / 4;                 // epilogue warps per lane quarter
+    const int wi = (warp - DEQ_WARP0) >> 2;            // this warp's index among them
+    const bool vec = (a.N % 8) == 0;
+    if (FMT != GEMM_BF16_SQ && a.splitk > 1) {
+      // split-K: store this CTA's fp32 partial tile; the CTA that arrives last at
+      // the tile's counter adds the splitk partials in split order and writes Y
+      // (no CTA waits for another; the sum's order does not depend on timing).
+      // Every epilogue warp passes both barriers, whether or not its wait succeeded.
       const float gmul = (FMT == GEMM_NVFP4) ? __ldg(a.gscale) : 1.0f;
-      const bool vec = (a.N % 8) == 0;
+      const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+      constexpr int TILE = BMT * BN;
+      if (go) {
+        tc_fence_after();
+        float* mine = a.part + (int64_t(tile) * a.splitk + blockIdx.z) * TILE;
+        for (int u = wi; u < S::NACC * (BN / 32); u += WPQ) {
+          const int acc = u / (BN / 32), c = (u % (BN / 32)) * 32;
+          const int rt = acc * kGemmBM + quarter * 32 + lane;  // row within the tile
+          uint32_t v[32];
+          tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN + c), v);
+          float4* dst = reinterpret_cast<float4*>(mine + rt * BN + c);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                 __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+        }
+      }
+      {
+        __threadfence();
+        asm volatile("bar.sync 1, %0;" ::"r"(DEQ_WARPS * 32) : "memory");  // the epilogue warps only
+        if (threadIdx.x == DEQ_WARP0 * 32)
+          *split_last = (atomicAdd(a.ctr + tile, 1u) == unsigned(a.splitk - 1)) ? 1 : 0;
+        asm volatile("bar.sync 1, %0;" ::"r"(DEQ_WARPS * 32) : "memory");
+        if (*split_last) {
+          __threadfence();
+          const float* base = a.part + int64_t(tile) * a.splitk * TILE;
+          for (int u = wi; u < S::NACC * (BN / 32); u += WPQ) {
+            const int acc = u / (BN / 32), c = (u % (BN / 32)) * 32;
+            const int rt = acc * kGemmBM + quarter * 32 + lane;
+            const int row = m0 + rt;
+            float v[32];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 x = __ldcg(reinterpret_cast<const float4*>(base + rt * BN + c) + q);
+              v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+            }
+            for (int sp = 1; sp < a.splitk; ++sp) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 x = __ldcg(reinterpret_cast<const float4*>(base + int64_t(sp) * TILE + rt * BN + c) + q);
+                v[4 * q] += x.x; v[4 * q + 1] += x.y; v[4 * q + 2] += x.z; v[4 * q + 3] += x.w;
+              }
+            }
+            if (row < a.M) {
+              uint16_t* yrow = a.Y + int64_t(row) * a.N;
+              const int nb = n0 + c;
+              if (vec && nb + 32 <= a.N) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  uint4 o;
+                  o.x = pack_bf16x2(v[8 * q + 0] * gmul, v[8 * q + 1] * gmul);
+                  o.y = pack_bf16x2(v[8 * q + 2] * gmul, v[8 * q + 3] * gmul);
+                  o.z = pack_bf16x2(v[8 * q + 4] * gmul, v[8 * q + 5] * gmul);
+                  o.w = pack_bf16x2(v[8 * q + 6] * gmul, v[8 * q + 7] * gmul);
+                  *reinterpret_cast<uint4*>(yrow + nb + 8 * q) = o;
+                }
+              } else {
+                for (int q = 0; q < 32; ++q)
+                  if (nb + q < a.N) yrow[nb + q] = uint16_t(f32_to_bf16_bits(v[q] * gmul));
+              }
+            }
+          }
+          if (threadIdx.x == DEQ_WARP0 * 32) a.ctr[tile] = 0u;  // clean for the next launch
+        }
+      }
+    } else if (go) {
+      tc_fence_after();
+      const float gmul = (FMT == GEMM_NVFP4) ? __ldg(a.gscale) : 1.0f;
       double sq = 0.0;
       // (accumulator, 32-column chunk) units of this quarter, dealt round-robin
       for (int u = wi; u < S::NACC * (BN / 32); u += WPQ) {

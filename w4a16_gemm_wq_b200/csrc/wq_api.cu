@@ -184,7 +184,7 @@ int launch_gemm_prepared(const wq::GemmArgs& a, cudaStream_t st) {
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((a.N + BN - 1) / BN, (a.M + BMT - 1) / BMT, 1);
+  cfg.gridDim = dim3((a.N + BN - 1) / BN, (a.M + BMT - 1) / BMT, a.splitk > 1 ? a.splitk : 1);
   cfg.blockDim = dim3(S::THREADS, 1, 1);
   cfg.dynamicSmemBytes = S::SMEM_BYTES;
   cfg.stream = st;
@@ -214,12 +214,63 @@ int gemm_bn(int64_t M, int64_t N);
 // dequantization, so one wave of them is never slower than two waves of
 // 128-row tiles: use it while it still covers about two thirds of the SMs,
 // with the widest W tile that does; else 128 rows.
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Plan of a quantized GEMM: the tile (see launch_gemm) and, when its CTAs
+// would cover under half of the SMs, how many CTAs share each output tile
+// along K (each at least 24 k-blocks) with the fp32 partials and per-tile
+// counters they need.
+struct GemmPlan {
+  int bn, bmt, splitk;
+  int64_t tiles;
+  size_t part_bytes, ws_bytes;
+};
+GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K) {
+  const auto tiles = [&](int bm, int bn) { return ((N + bn - 1) / bn) * ((M + bm - 1) / bm); };
+  GemmPlan p = {};
+  if (tiles(256, 256) >= 100) {
+    p.bn = 256; p.bmt = 256;
+  } else if (tiles(256, 128) >= 100) {
+    p.bn = 128; p.bmt = 256;
+  } else {
+    p.bn = gemm_bn(M, N); p.bmt = wq::kGemmBM;
+  }
+  p.tiles = tiles(p.bmt, p.bn);
+  const int64_t nkb = (K + wq::kGemmBK - 1) / wq::kGemmBK;
+  int64_t s = 1;
+  // at least 24 k-blocks per CTA: shorter K ranges lose more to the per-CTA start
+  // and the partial traffic than they gain (measured: K = 2048 slower split)
+  if (p.tiles < wq::kTcMaxCtas / 2) s = std::max<int64_t>(1, std::min<int64_t>({wq::kTcMaxCtas / p.tiles, 8, nkb / 24}));
+  p.splitk = int(s);
+  p.part_bytes = s > 1 ? align256(size_t(p.tiles) * size_t(s) * size_t(p.bmt) * size_t(p.bn) * 4) : 0;
+  p.ws_bytes = s > 1 ? p.part_bytes + align256(size_t(p.tiles) * 4) : 0;
+  return p;
+}
+
+// Tile of the quantized GEMM.  A 256-row CTA (two accumulators sharing each
+// dequantized W tile) does twice the flops of a 128-row one for the same
+// dequantization, so one wave of them is never slower than two waves of
+// 128-row tiles: use it while it still covers about two thirds of the SMs,
+// with the widest W tile that does; else 128 rows.  Few tiles (under half the
+// SMs) split K over several CTAs per tile when the caller's workspace holds
+// the partials.
 template <int FMT>
-int launch_gemm(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaStream_t st) {
-  const auto tiles = [&](int bm, int bn) { return ((a.N + bn - 1) / bn) * int64_t((a.M + bm - 1) / bm); };
-  if (tiles(256, 256) >= 100) return launch_gemm_bn<FMT, 256, 256>(a, X, packed, st);
-  if (tiles(256, 128) >= 100) return launch_gemm_bn<FMT, 128, 256>(a, X, packed, st);
-  if (gemm_bn(a.M, a.N) == 256) return launch_gemm_bn<FMT, 256>(a, X, packed, st);
+int launch_gemm(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaStream_t st, void* ws = nullptr,
+                size_t ws_bytes = 0) {
+  const GemmPlan p = gemm_plan(a.M, a.N, a.K);
+  a.splitk = 1;
+  if (p.splitk > 1 && ws && ws_bytes >= p.ws_bytes && aligned16(ws)) {
+    a.splitk = p.splitk;
+    a.part = static_cast<float*>(ws);
+    a.ctr = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + p.part_bytes);
+    // the kernel leaves the counters at 0, but the workspace may be fresh memory
+    if (int e = cuda_check(cudaMemsetAsync(a.ctr, 0, size_t(p.tiles) * 4, st), "split-K counters")) return e;
+  }
+  if (p.bmt == 256) {
+    if (p.bn == 256) return launch_gemm_bn<FMT, 256, 256>(a, X, packed, st);
+    return launch_gemm_bn<FMT, 128, 256>(a, X, packed, st);
+  }
+  if (p.bn == 256) return launch_gemm_bn<FMT, 256>(a, X, packed, st);
   return launch_gemm_bn<FMT, 128>(a, X, packed, st);
 }
 
@@ -227,8 +278,6 @@ int gemm_bn(int64_t M, int64_t N) {
   const int64_t tiles256 = int64_t((N + 255) / 256) * ((M + wq::kGemmBM - 1) / wq::kGemmBM);
   return tiles256 >= 148 ? 256 : 128;
 }
-
-size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Workspace of awq_search_scale: a (fp64 [K]), s (fp32 [K]), loss partials
 // (fp64 [n_alpha, P]) and, with calibration tokens, Delta (bf16 [N, 2K]).
@@ -654,7 +703,7 @@ int wq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int format, int ac
   if (act_fp4) {
     *bytes = w4a4_layout(M, K).total;
   } else {
-    *bytes = 0;
+    *bytes = M > kGemvMaxM ? gemm_plan(M, N, K).ws_bytes : 0;
   }
   return WQ_OK;
 }
@@ -847,8 +896,6 @@ int awq_search_scale_shared(const uint16_t* const* Ws, const int64_t* Ns, int n_
 int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* qweight,
                    const uint16_t* scales, const uint32_t* zeros, int group_size, int zero_point,
                    const float* act_inv_s, uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   REQUIRE(M > 0 && M <= (int64_t(1) << 30), "M must be positive");
   if (int e = check_shape(N, K)) return e;
   if (int e = check_group(group_size, K)) return e;
@@ -867,7 +914,7 @@ int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uin
     wq::GemmArgs g = {};
     g.scales = scales; g.zeros = zeros; g.inv_s = act_inv_s; g.Y = Y;
     g.M = int(M); g.N = int(N); g.K = int(K); g.log2g = log2i(group_size);
-    return launch_gemm<wq::FMT_INT4>(g, X, qweight, as_stream(stream));
+    return launch_gemm<wq::FMT_INT4>(g, X, qweight, as_stream(stream), ws, ws_bytes);
   }
   wq::GemvArgs a = {};
   a.X = X; a.inv_s = act_inv_s; a.wq = qweight; a.scales = scales; a.zeros = zeros;
@@ -907,7 +954,7 @@ int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const ui
     wq::GemmArgs g = {};
     g.bscale = bscale; g.gscale = global_scale; g.inv_s = act_inv_s; g.Y = Y;
     g.M = int(M); g.N = int(N); g.K = int(K);
-    return launch_gemm<wq::FMT_NVFP4>(g, X, codes, as_stream(stream));
+    return launch_gemm<wq::FMT_NVFP4>(g, X, codes, as_stream(stream), ws, ws_bytes);
   }
   wq::GemvArgs a = {};
   a.X = X; a.inv_s = act_inv_s; a.wq = codes; a.bscale = bscale; a.gscale = global_scale;
