@@ -40,6 +40,7 @@ namespace wq {
 constexpr int kGptqThreads = 512;  // 16 warps
 constexpr int kGptqMaxRows = 16;   // rows per pass: one warp each in the sequential part
 
+
 struct GptqArgs {
   const uint16_t* W;   // bf16 [N, K]
   const float* U;      // fp32 [K, K], upper triangle read
@@ -55,8 +56,11 @@ __host__ __device__ inline size_t gptq_smem_bytes(int R, int64_t K, int G) {
   return size_t(R) * size_t(K) * 4 + size_t(G) * G * 4 + size_t(R) * G * 4 + size_t(R) * G;
 }
 
-template <int G, bool ASYM>
+// RMAX: the largest row count of a pass this instantiation serves (4 for long
+// rows, where U streams from DRAM and more loads in flight pay; 16 otherwise).
+template <int G, bool ASYM, int RMAX>
 __global__ void __launch_bounds__(kGptqThreads, 1) gptq_int4_kernel(const GptqArgs a) {
+  constexpr int UCHUNK = RMAX <= 4 ? 32 : 16;  // U loads in flight per thread in the update part
   extern __shared__ __align__(16) float gsm[];
   const int R = a.R;
   const int64_t K = a.K;
@@ -162,27 +166,32 @@ __global__ void __launch_bounds__(kGptqThreads, 1) gptq_int4_kernel(const GptqAr
 
       // ---- 3. the block's errors applied to the later columns, k in order
       for (int64_t j = b + G + threadIdx.x; j < K; j += kGptqThreads) {
-        float acc[kGptqMaxRows];
+        float acc[RMAX];
 #pragma unroll
-        for (int r = 0; r < kGptqMaxRows; ++r)
+        for (int r = 0; r < RMAX; ++r)
           if (r < rows) acc[r] = w[int64_t(r) * K + j];
         const float* uc = a.U + b * K + j;
-#pragma unroll 2
-        for (int kk = 0; kk < G; kk += 4) {  // four k per step: one 16-byte error load per row
-          const float u0 = __ldg(uc + int64_t(kk) * K), u1 = __ldg(uc + int64_t(kk + 1) * K);
-          const float u2 = __ldg(uc + int64_t(kk + 2) * K), u3 = __ldg(uc + int64_t(kk + 3) * K);
+        for (int k0 = 0; k0 < G; k0 += UCHUNK) {
+          // a chunk of U's column j in flight at once (the loads, not the FMAs,
+          // bound this loop when U streams from L2 or DRAM)
+          float u[UCHUNK];
 #pragma unroll
-          for (int r = 0; r < kGptqMaxRows; ++r)
-            if (r < rows) {
-              const float4 ne = *reinterpret_cast<const float4*>(errs + r * G + kk);
-              acc[r] = __fmaf_rn(ne.x, u0, acc[r]);
-              acc[r] = __fmaf_rn(ne.y, u1, acc[r]);
-              acc[r] = __fmaf_rn(ne.z, u2, acc[r]);
-              acc[r] = __fmaf_rn(ne.w, u3, acc[r]);
-            }
+          for (int q = 0; q < UCHUNK; ++q) u[q] = __ldg(uc + int64_t(k0 + q) * K);
+#pragma unroll
+          for (int q = 0; q < UCHUNK; q += 4) {  // four k per step: one 16-byte error load per row
+#pragma unroll
+            for (int r = 0; r < RMAX; ++r)
+              if (r < rows) {
+                const float4 ne = *reinterpret_cast<const float4*>(errs + r * G + k0 + q);
+                acc[r] = __fmaf_rn(ne.x, u[q], acc[r]);
+                acc[r] = __fmaf_rn(ne.y, u[q + 1], acc[r]);
+                acc[r] = __fmaf_rn(ne.z, u[q + 2], acc[r]);
+                acc[r] = __fmaf_rn(ne.w, u[q + 3], acc[r]);
+              }
+          }
         }
 #pragma unroll
-        for (int r = 0; r < kGptqMaxRows; ++r)
+        for (int r = 0; r < RMAX; ++r)
           if (r < rows) w[int64_t(r) * K + j] = acc[r];
       }
       __syncthreads();

@@ -784,8 +784,12 @@ int wq_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int gr
     kern<<<grid, wq::kGptqThreads, smem, st>>>(a);
     return launched("gptq_int4 launch");
   };
-  if (G == 64) return zero_point ? go(wq::gptq_int4_kernel<64, true>) : go(wq::gptq_int4_kernel<64, false>);
-  return zero_point ? go(wq::gptq_int4_kernel<128, true>) : go(wq::gptq_int4_kernel<128, false>);
+  if (R <= 4) {
+    if (G == 64) return zero_point ? go(wq::gptq_int4_kernel<64, true, 4>) : go(wq::gptq_int4_kernel<64, false, 4>);
+    return zero_point ? go(wq::gptq_int4_kernel<128, true, 4>) : go(wq::gptq_int4_kernel<128, false, 4>);
+  }
+  if (G == 64) return zero_point ? go(wq::gptq_int4_kernel<64, true, 16>) : go(wq::gptq_int4_kernel<64, false, 16>);
+  return zero_point ? go(wq::gptq_int4_kernel<128, true, 16>) : go(wq::gptq_int4_kernel<128, false, 16>);
 }
 
 int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scale_s, uint8_t* codes,
