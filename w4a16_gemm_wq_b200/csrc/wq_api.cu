@@ -770,7 +770,7 @@ int wq_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int gr
     return e;
   if (int e = cuda_check(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "SM count")) return e;
   const int G = group_size;
-  const int64_t fit = (int64_t(optin) - int64_t(G) * G * 4) / (K * 4 + int64_t(G) * 5);
+  const int64_t fit = (int64_t(optin) - int64_t(G) * G * 4 - int64_t(G) * 4) / (K * 4 + int64_t(G) * 5);
   const int R = int(std::min<int64_t>({int64_t(wq::kGptqMaxRows), N, fit}));
   if (R < 1) return fail(WQ_ERR_UNSUPPORTED, "K = %lld is too long for one row in shared memory", (long long)K);
   wq::GptqArgs a = {W, U, N, K, R, qweight, scales, zeros};
