@@ -133,16 +133,16 @@ __global__ void __launch_bounds__(kGptqThreads, 1) gptq_int4_kernel(const GptqAr
 #pragma unroll
             for (int i2 = 0; i2 < PL; ++i2) urow[i2] = ud[kk * G + lane + 32 * i2];
             const float rk = dinv[kk];
-            float e = 0.0f;
-            if (lane == l2) {  // the lane holding column kk quantizes it
-              const float q = ASYM ? fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(v[i], sc)), z), 0.0f), 15.0f)
-                                   : __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(v[i], sc)), -7.0f), 7.0f), 8.0f);
-              const float deq = __fmul_rn(__fsub_rn(q, z), sc);  // exact: |q - z| <= 15, sc has 11 bits
-              e = __fmul_rn(__fsub_rn(v[i], deq), rk);
+            // every lane quantizes its own column of slot i (no divergent branch);
+            // the lane holding column kk keeps its code and error, all take its error
+            const float q = ASYM ? fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(v[i], sc)), z), 0.0f), 15.0f)
+                                 : __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(v[i], sc)), -7.0f), 7.0f), 8.0f);
+            const float deq = __fmul_rn(__fsub_rn(q, z), sc);  // exact: |q - z| <= 15, sc has 11 bits
+            const float e = __shfl_sync(0xFFFFFFFFu, __fmul_rn(__fsub_rn(v[i], deq), rk), l2);
+            if (lane == l2) {
               qb[warp * G + kk] = uint8_t(q);
               errs[warp * G + kk] = -e;
             }
-            e = __shfl_sync(0xFFFFFFFFu, e, l2);
 #pragma unroll
             for (int i2 = 0; i2 < PL; ++i2) {
               const int jj = lane + 32 * i2;
