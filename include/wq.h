@@ -62,7 +62,7 @@ typedef enum {
   WQ_OK = 0,
   WQ_ERR_ARG = 1,         /* null/misaligned pointer, bad size, too-small workspace */
   WQ_ERR_CUDA = 2,        /* a CUDA launch or runtime call failed */
-  WQ_ERR_UNSUPPORTED = 3, /* bits != 4, group_size not in {64, 128}, ... */
+  WQ_ERR_UNSUPPORTED = 3, /* bits != 4, group_size not in {32, 64, 128}, ... */
   WQ_ERR_TIMEOUT = 4      /* a device-side bounded wait gave up (see wq_device_error) */
 } wq_status;
 
@@ -100,7 +100,7 @@ int awq_search_workspace_size(int64_t N, int64_t K, int64_t T, int n_alpha, int 
  * sections 2-3; "Lance-Quant" section "量化应用": pack by group).
  *   W        bf16 [N, K]
  *   bits     must be 4
- *   group_size 64 or 128 (K % group_size == 0)
+ *   group_size 32, 64 or 128 (K % group_size == 0)
  *   zero_point 1 = asymmetric with per-group zero point, 0 = symmetric
  *   scale_s  fp32 [K] AWQ per-input-channel scale, or NULL; when given the
  *            library quantizes w' = W[n,k] * scale_s[k] (fp32 multiply)
@@ -237,7 +237,7 @@ typedef struct {
   const void* packed;         /* INT4 qweight (uint32 [N, K/8]) or NVFP4 codes (uint8 [N, K/2]) */
   const uint16_t* scales;     /* INT4 fp16 [N, K/G] */
   const uint32_t* zeros;      /* INT4 packed zero points, NULL for a symmetric pack */
-  int group_size;             /* INT4: 64 or 128 */
+  int group_size;             /* INT4: 32, 64 or 128 (32 runs the CUDA-core GEMV) */
   int zero_point;             /* INT4: 1 asymmetric, 0 symmetric */
   const uint8_t* bscale;      /* NVFP4 E4M3 [N, K/16] */
   const float* global_scale;  /* NVFP4 fp32 [1] */

@@ -44,8 +44,9 @@ def test_size_queries(lib):
     with pytest.raises(wq.WQError) as e:
         wq.int4_sizes(16, 100, 64)  # K not a multiple of 32
     assert e.value.status == wq.WQ_ERR_ARG
+    assert wq.int4_sizes(16, 512, 32) == (16 * 256, 16 * 16 * 2, 16 * 2 * 4)
     with pytest.raises(wq.WQError) as e:
-        wq.int4_sizes(16, 512, 32)
+        wq.int4_sizes(16, 512, 256)
     assert e.value.status == wq.WQ_ERR_UNSUPPORTED
 
 

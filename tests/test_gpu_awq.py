@@ -32,7 +32,7 @@ def _ulps(a, b):
     return np.max(np.abs(a.view(np.int32).astype(np.int64) - b.view(np.int32).astype(np.int64)))
 
 
-@pytest.mark.parametrize("G", [64, 128])
+@pytest.mark.parametrize("G", [32, 64, 128])
 @pytest.mark.parametrize("N,K,T", [(48, 256, 64), (200, 1024, 130), (256, 512, 512)])
 def test_search_with_tokens_small(lib, G, N, K, T):
     W = synth.weight(N, K, seed=N + K, outlier_frac=0.02)

@@ -25,7 +25,7 @@ def _deq(p):
 
 
 @pytest.mark.parametrize("M", [17, 64, 128, 129, 200, 512])
-@pytest.mark.parametrize("fmt", ["int4_g64", "int4_g128", "int4_sym", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["int4_g64", "int4_g128", "int4_g32", "int4_sym", "nvfp4"])
 def test_small_gemm_all_rows(lib, M, fmt):
     K, N = 512, 384  # 3 N-tiles of 128, ragged M tiles
     W = synth.weight(N, K, seed=M)
@@ -35,7 +35,7 @@ def test_small_gemm_all_rows(lib, M, fmt):
         Y = lib.wq_linear_nvfp4(X.cuda(), p)
         ref = _ref_nvfp4(p, X)
     else:
-        G = 128 if fmt == "int4_g128" else 64
+        G = {"int4_g128": 128, "int4_g32": 32}.get(fmt, 64)
         p = lib.wq_quantize_int4(W.cuda(), G, 0 if fmt == "int4_sym" else 1)
         Y = lib.wq_linear_int4(X.cuda(), p)
         ref = _ref_int4(p, X)

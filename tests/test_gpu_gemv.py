@@ -41,7 +41,7 @@ def test_config1_awq_m1_m16(lib):
 
 
 @pytest.mark.parametrize("K,N", synth.DECODE_SHAPES)
-@pytest.mark.parametrize("fmt", ["int4_g128", "int4_g64", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["int4_g128", "int4_g64", "int4_g32", "nvfp4"])
 def test_config2_decode_m1(lib, K, N, fmt):
     W = synth.weight(N, K, seed=synth.layer_seed(2, K + N))
     X = synth.activations(1, K, seed=synth.layer_seed(2, K))

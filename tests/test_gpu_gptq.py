@@ -30,7 +30,7 @@ def _check(p, ref, rows=None):
         np.testing.assert_array_equal(g if rows is None else g[rows], ref[name], err_msg=name)
 
 
-@pytest.mark.parametrize("G", [64, 128])
+@pytest.mark.parametrize("G", [32, 64, 128])
 @pytest.mark.parametrize("zp", [1, 0])
 @pytest.mark.parametrize("N,K", [(37, 256), (16, 1024), (100, 512)])
 def test_gptq_bit_exact(lib, G, zp, N, K):

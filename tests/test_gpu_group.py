@@ -54,7 +54,7 @@ def test_decode_sweep_group(lib, M):
 def test_ragged_shapes_scales_and_symmetric(lib):
     M = 1
     shapes = [(96, 40, "nvfp4"), (1088, 200, "int4_g64"), (2048, 17, "int4_sym"), (11008, 33, "nvfp4"),
-              (512, 16, "int4_g128"), (3072, 1, "int4_g64")]
+              (512, 16, "int4_g128"), (3072, 1, "int4_g64"), (2048, 96, "int4_g32")]
     items = []
     for i, (K, N, fmt) in enumerate(shapes):
         W = synth.weight(N, K, seed=100 + i)

@@ -46,7 +46,7 @@ def test_config1_awq_int4_g64(lib):
 
 
 @pytest.mark.parametrize("K,N", synth.DECODE_SHAPES)
-@pytest.mark.parametrize("G", [128, 64])
+@pytest.mark.parametrize("G", [128, 64, 32])
 def test_config2_int4_shapes(lib, K, N, G):
     W = synth.weight(N, K, seed=synth.layer_seed(2, K + N))
     _check_int4(lib, W, G)

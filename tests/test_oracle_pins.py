@@ -156,7 +156,7 @@ def test_int4_symmetric_example():
     assert deq[0] == 7 * sc and deq[1] == -7 * sc and deq[2] == 0.0
 
 
-@pytest.mark.parametrize("G", [64, 128])
+@pytest.mark.parametrize("G", [32, 64, 128])
 def test_int4_round_trip_bound_and_brute_force(G):
     N, K = 48, 512
     W = synth.weight(N, K, seed=11)

@@ -349,6 +349,8 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
       if (FMT == GEMM_INT4) {
         const int g = (kb * kGemmBK) >> a.log2g;
         raw_a = __ldg(a.scales + int64_t(n) * ng + g);
+        if (a.log2g == 5 && g + 1 < ng)  // G = 32: the k-block's second group (same zero word: g is even)
+          raw_a |= uint32_t(__ldg(a.scales + int64_t(n) * ng + g + 1)) << 16;
         if (a.zeros) raw_b = __ldg(a.zeros + int64_t(n) * zw_stride + (g >> 3));
       } else if (FMT == GEMM_NVFP4) {
         const int nb = a.K >> 4;
@@ -368,15 +370,19 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
       const int kb = kbeg + i, s = i % STAGES, r = i / STAGES;
       const uint32_t cur_a = meta_a, cur_b = meta_b;
       fetch_meta(kb + 1, meta_a, meta_b);
-      uint32_t sc2 = 0, zoff2 = 0;
+      uint32_t sc2[2] = {0, 0}, zoff2[2] = {0, 0};  // INT4: words 0-3 / 4-7 (two groups when G = 32)
       uint32_t sbv[4] = {0, 0, 0, 0};  // NVFP4: the k-block's 4 E4M3 block scales as bf16x2 {sb, sb}
       if (FMT == GEMM_INT4) {
         const int g = (kb * kGemmBK) >> a.log2g;
-        const float sc = __half2float(__ushort_as_half(uint16_t(cur_a)));
-        const int z = (cur_b >> (4 * (g & 7))) & 0xF;
-        sc2 = pack_bf16x2(sc, sc);
-        const uint32_t zb = 0x4300u | uint32_t(z);  // bf16(128 + z)
-        zoff2 = zb | (zb << 16);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int gh = g + (a.log2g == 5 ? h : 0);
+          const float sc = __half2float(__ushort_as_half(uint16_t(a.log2g == 5 && h ? cur_a >> 16 : cur_a)));
+          const int z = (cur_b >> (4 * (gh & 7))) & 0xF;
+          sc2[h] = pack_bf16x2(sc, sc);
+          const uint32_t zb = 0x4300u | uint32_t(z);  // bf16(128 + z)
+          zoff2[h] = zb | (zb << 16);
+        }
       } else {
 #pragma unroll
         for (int q = 0; q < 4; q += 2) {  // two E4M3 bytes -> f16x2 -> fp32 -> bf16 (all exact), then replicate each
@@ -395,7 +401,8 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
       const uint32_t brow = b_addr(s);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        uint4 v = (FMT == GEMM_INT4) ? dequant_word_int4(words[j], zoff2, sc2) : dequant_word_nvfp4(words[j], sbv[j >> 1]);
+        uint4 v = (FMT == GEMM_INT4) ? dequant_word_int4(words[j], zoff2[j >> 2], sc2[j >> 2])
+                                     : dequant_word_nvfp4(words[j], sbv[j >> 1]);
         if (a.inv_s) {
           const int k = kb * kGemmBK + 8 * j;
           if (k < a.K) {

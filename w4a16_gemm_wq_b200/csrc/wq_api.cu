@@ -65,8 +65,8 @@ int check_shape(int64_t N, int64_t K) {
 }
 
 int check_group(int group_size, int64_t K) {
-  if (group_size != 64 && group_size != 128)
-    return fail(WQ_ERR_UNSUPPORTED, "group_size must be 64 or 128 (got %d)", group_size);
+  if (group_size != 32 && group_size != 64 && group_size != 128)
+    return fail(WQ_ERR_UNSUPPORTED, "group_size must be 32, 64 or 128 (got %d)", group_size);
   REQUIRE(K % group_size == 0, "K (%lld) must be a multiple of group_size (%d)", (long long)K, group_size);
   return WQ_OK;
 }
@@ -434,6 +434,7 @@ int tc_kind(const TcCall& c, int64_t M) {
   const auto a4 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 3) == 0; };
   if (c.fmt == wq::FMT_INT4) {
     if (!a4(c.scales) || (c.zeros && !a4(c.zeros))) return -1;
+    if (c.group_size != 64 && c.group_size != 128) return -1;  // G = 32: the CUDA-core GEMV serves it
     return c.group_size == 64 ? wq::TC_INT4_G64 : wq::TC_INT4_G128;
   }
   if (!a4(c.bscale)) return -1;
@@ -735,7 +736,12 @@ int wq_quantize_int4(const uint16_t* W, int64_t N, int64_t K, int bits, int grou
   }
   const dim3 grid(unsigned((K / 8 + wq::kQuantThreads - 1) / wq::kQuantThreads), unsigned(N));
   cudaStream_t st = as_stream(stream);
-  if (group_size == 64) {
+  if (group_size == 32) {
+    if (zero_point)
+      wq::quantize_int4_kernel<32, true><<<grid, wq::kQuantThreads, 0, st>>>(W, scale_s, N, K, qweight, scales, zeros);
+    else
+      wq::quantize_int4_kernel<32, false><<<grid, wq::kQuantThreads, 0, st>>>(W, scale_s, N, K, qweight, scales, zeros);
+  } else if (group_size == 64) {
     if (zero_point)
       wq::quantize_int4_kernel<64, true><<<grid, wq::kQuantThreads, 0, st>>>(W, scale_s, N, K, qweight, scales, zeros);
     else
@@ -785,9 +791,11 @@ int wq_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int gr
     return launched("gptq_int4 launch");
   };
   if (R <= 4) {
+    if (G == 32) return zero_point ? go(wq::gptq_int4_kernel<32, true, 4>) : go(wq::gptq_int4_kernel<32, false, 4>);
     if (G == 64) return zero_point ? go(wq::gptq_int4_kernel<64, true, 4>) : go(wq::gptq_int4_kernel<64, false, 4>);
     return zero_point ? go(wq::gptq_int4_kernel<128, true, 4>) : go(wq::gptq_int4_kernel<128, false, 4>);
   }
+  if (G == 32) return zero_point ? go(wq::gptq_int4_kernel<32, true, 16>) : go(wq::gptq_int4_kernel<32, false, 16>);
   if (G == 64) return zero_point ? go(wq::gptq_int4_kernel<64, true, 16>) : go(wq::gptq_int4_kernel<64, false, 16>);
   return zero_point ? go(wq::gptq_int4_kernel<128, true, 16>) : go(wq::gptq_int4_kernel<128, false, 16>);
 }
@@ -864,7 +872,9 @@ static int awq_search_pieces(const uint16_t* const* Ws, const int64_t* Ns, int n
       const dim3 dgrid(gx, unsigned(Ns[p]));
       uint16_t* Dp = D ? D + row * 2 * K : nullptr;
       double* pp = D ? part_i : part_i + row * gx;  // proxy partials: one per (row, CTA column)
-      if (group_size == 64)
+      if (group_size == 32)
+        wq::awq_delta_kernel<32><<<dgrid, wq::kQuantThreads, 0, st>>>(Ws[p], s, Ns[p], K, Dp, a, pp);
+      else if (group_size == 64)
         wq::awq_delta_kernel<64><<<dgrid, wq::kQuantThreads, 0, st>>>(Ws[p], s, Ns[p], K, Dp, a, pp);
       else
         wq::awq_delta_kernel<128><<<dgrid, wq::kQuantThreads, 0, st>>>(Ws[p], s, Ns[p], K, Dp, a, pp);
