@@ -465,7 +465,8 @@ def prefill_measure(wq, synth, torch, dev, peaks, Ms=(512, 2048, 8192), reps=20,
 
 def quant_measure(wq, synth, torch, dev, peaks, reps=10):
     """Stage-1 throughput on the 7 projections of one block: INT4 g64 with an
-    AWQ scale, and NVFP4.  GB/s counts bf16 weights read + packed bytes written."""
+    AWQ scale, and NVFP4, replayed from a CUDA graph of the block's launches.
+    GB/s counts bf16 weights read + packed bytes written."""
     Ws = [synth.weight(N, K, seed=synth.layer_seed(5, i), device=dev) for i, (_, K, N) in enumerate(synth.PROJECTIONS)]
     Ss = [synth.act_mean_lognormal(W.shape[1], seed=i, device=dev).sqrt() for i, W in enumerate(Ws)]
     out = {}
@@ -482,13 +483,20 @@ def quant_measure(wq, synth, torch, dev, peaks, reps=10):
         for W in Ws:
             N, K = W.shape
             nbytes += 2 * N * K + (N * K // 2 + N * K // 16 if fmt == "nvfp4" else sum(wq.int4_sizes(N, K, 64)))
+        # the block's launches captured once (device time only, as for the linears)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run()
+        g.replay()
+        torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         for _ in range(reps):
-            run()
+            g.replay()
         b.record()
         torch.cuda.synchronize()
         sec = a.elapsed_time(b) * 1e-3 / reps
+        del g
         out[fmt] = {"GB/s": round(nbytes / sec / 1e9, 1), "frac_of_hbm": round(nbytes / sec / 1e9 / peaks["hbm"], 4),
                     "us_per_block": round(sec * 1e6, 1)}
     return out
