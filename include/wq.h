@@ -250,11 +250,12 @@ typedef struct {
  * primer" section 13: decode is memory-bound, so the weights must stream at
  * HBM speed; one launch pays the launch and ramp cost once for the whole
  * group).  Each item's Y is what its single entry point computes.  At M <= 2
- * the items the tensor-core decode GEMV serves (K % 128 == 0, 16-byte aligned
- * X / packed / act_inv_s, 4-byte aligned scale data) run as one launch per
- * kernel variant (INT4 group 64, INT4 group 128, NVFP4), up to 24 items and 8
- * distinct activation vectors each; the other items run one by one after
- * them.  Items must not alias each other's outputs.  Needs no workspace.
+ * the items the tensor-core decode GEMV serves (K % 128 == 0, INT4 group 64
+ * or 128 or NVFP4, 16-byte aligned X / packed / act_inv_s, 4-byte aligned
+ * scale data) run as one launch for all their weight kinds together, up to 24
+ * items and 8 distinct activation vectors; the other items (M > 2, group 32,
+ * other K) run one by one after them.  Items must not alias each other's
+ * outputs.  Needs no workspace.
  * Returns the first failing item's status. */
 int wq_linear_group(const wq_linear_item* items, int count, int64_t M, void* stream);
 

@@ -13,7 +13,7 @@
 // kTcDepth steps (3 KB) in flight in registers.
 //
 // Partition: CTA b owns the row blocks [bounds[b], bounds[b+1]) of the
-// launch (items in order, balanced by bytes on the host); its 8 warps split
+// launch (items in order, balanced by time on the host); its 16 warps split
 // the CTA's steps evenly (stream-K inside the CTA).  A row block inside one
 // warp's range is written directly; one split over warps leaves an fp32
 // partial per warp in shared memory, and the warp that arrives last (shared
