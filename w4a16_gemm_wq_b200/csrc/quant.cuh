@@ -129,55 +129,52 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_int4_kernel(
   }
 }
 
-// ------------------------------------------------------------------ NVFP4
-// Round-to-nearest-even of a non-negative finite fp32 to E4M3, saturating
-// at 448 (code 0x7E).  Bit-level rounding of the fp32 significand.
-__device__ __forceinline__ uint32_t e4m3_encode_satfinite(float t) {
-  if (!(t < 448.0f)) return 0x7E;          // also catches +inf
-  const uint32_t bits = __float_as_uint(t);
-  const int E = int(bits >> 23) - 127;
-  if (E < -6) {                            // below 2^-6: subnormal grid m * 2^-9
-    const float m = rintf(t * 512.0f);       // exact scaling, RNE
-    return uint32_t(m);                      // m == 8 encodes 2^-6 = code 0x08
+// 8 consecutive elements at flat index e of a row-major [R, C] bf16 tensor as
+// fp32, times s[e % C] when an AWQ scale is given (the column is only needed then).
+__device__ __forceinline__ void load_flat8(const uint16_t* __restrict__ A, const float* __restrict__ s, int64_t C,
+                                           int64_t e, float w[8]) {
+  const uint4 v = ldg_stream_v4(A + e);
+  const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    w[2 * j] = __uint_as_float(u[j] << 16);
+    w[2 * j + 1] = __uint_as_float(u[j] & 0xFFFF0000u);
   }
-  uint32_t e = uint32_t(E + 7);
-  const uint32_t man = bits & 0x7FFFFFu;
-  uint32_t keep = man >> 20;
-  const uint32_t rem = man & 0xFFFFFu;
-  if (rem > 0x80000u || (rem == 0x80000u && (keep & 1u))) ++keep;
-  if (keep == 8) { keep = 0; ++e; }
-  if (e > 15 || (e == 15 && keep == 7)) return 0x7E;
-  return (e << 3) | keep;
+  if (s) {
+    const int64_t c = e % C;
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + c));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + c + 4));
+    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = __fmul_rn(w[j], sv[j]);
+  }
 }
 
-// Nearest E2M1 code of v (ties to the even code, saturating at 6, sign bit
-// from v).  Magnitudes by code: 0, 0.5, 1, 1.5, 2, 3, 4, 6.
-__device__ __forceinline__ uint32_t e2m1_encode(float v) {
-  const float a = fabsf(v);
-  uint32_t c;
-  if (a <= 0.25f) c = 0;
-  else if (a < 0.75f) c = 1;
-  else if (a <= 1.25f) c = 2;
-  else if (a < 1.75f) c = 3;
-  else if (a <= 2.5f) c = 4;
-  else if (a < 3.5f) c = 5;
-  else if (a <= 5.0f) c = 6;
-  else c = 7;
-  return c | ((__float_as_uint(v) >> 28) & 8u);
-}
-
+// ------------------------------------------------------------------ NVFP4
 // Pass 1: amax over the tensor, atomically max-ed into *amax_out (which the
 // host zeroed).  Non-negative floats order like their bit patterns.
 __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const uint16_t* __restrict__ A, const float* __restrict__ s,
                                                          int64_t R, int64_t C, float* amax_out) {
   const int64_t words = R * C / 8;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
   float m = 0.f;
-  for (int64_t u = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u < words; u += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = (u * 8) / C, c = (u * 8) % C;
-    float w[8];
-    load_wprime8(A, s, C, r, c, w);
+  // four independent 16-byte loads in flight per thread per iteration
+  for (int64_t u0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u0 < words; u0 += 4 * stride) {
+    float w[4][8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(w[j]));
+    for (int q = 0; q < 4; ++q) {
+      const int64_t u = u0 + q * stride;
+      if (u < words) {
+        load_flat8(A, s, C, u * 8, w[q]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[q][j] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(w[q][j]));
   }
 #pragma unroll
   for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -188,6 +185,24 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const uint16_t* __restr
     for (int i = 1; i < int(blockDim.x >> 5); ++i) m = fmaxf(m, red[i]);
     atomicMax(reinterpret_cast<unsigned int*>(amax_out), __float_as_uint(m));
   }
+}
+
+// Hardware conversions: round to nearest with ties to the even mantissa (for
+// E2M1 that is the even code), saturating at the largest finite value, sign
+// kept -- the readings of the pages' "E2M1 + E4M3" packing; the bit-exact pack
+// tests hold them to the oracle's table-driven encoders, exact ties and both
+// signs included.
+// Two fp32 -> E2M1 codes, `lo` in bits 0-3 and `hi` in bits 4-7.
+__device__ __forceinline__ uint32_t e2m1x2_rn_sat(float lo, float hi) {
+  uint32_t d;
+  asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u32.u8 %0, t; }" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+// One non-negative fp32 -> E4M3 code (satfinite: 448 for anything larger).
+__device__ __forceinline__ uint32_t e4m3_rn_sat(float t) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(0.0f), "f"(t));
+  return uint32_t(d) & 0xFFu;
 }
 
 __device__ __forceinline__ float nvfp4_global_from_amax(float amax) {
@@ -202,23 +217,25 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(const uint16_t* __restr
   const int64_t nblk = R * C / 16;
   const float g = nvfp4_global_from_amax(*amax_in);
   for (int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; b < nblk; b += int64_t(gridDim.x) * blockDim.x) {
-    const int64_t r = (b * 16) / C, c = (b * 16) % C;
     float w[16];
-    load_wprime8(A, s, C, r, c, w);
-    load_wprime8(A, s, C, r, c + 8, w + 8);
+    load_flat8(A, s, C, b * 16, w);
+    load_flat8(A, s, C, b * 16 + 8, w + 8);
     float ab = 0.f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) ab = fmaxf(ab, fabsf(w[j]));
     const float t = __fdiv_rn(__fdiv_rn(ab, 6.0f), g);
-    const uint32_t sb = e4m3_encode_satfinite(t);
+    const uint32_t sb = e4m3_rn_sat(t);
     const float d = e4m3_decode_pos(sb);
     uint32_t lo = 0, hi = 0;
     if (d != 0.0f) {
       const float denom = __fmul_rn(d, g);
+      // the IEEE quotient, then two codes per conversion instruction
 #pragma unroll
-      for (int j = 0; j < 8; ++j) lo |= e2m1_encode(__fdiv_rn(w[j], denom)) << (4 * j);
+      for (int j = 0; j < 8; j += 2)
+        lo |= e2m1x2_rn_sat(__fdiv_rn(w[j], denom), __fdiv_rn(w[j + 1], denom)) << (4 * j);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) hi |= e2m1_encode(__fdiv_rn(w[8 + j], denom)) << (4 * j);
+      for (int j = 0; j < 8; j += 2)
+        hi |= e2m1x2_rn_sat(__fdiv_rn(w[8 + j], denom), __fdiv_rn(w[9 + j], denom)) << (4 * j);
     }
     reinterpret_cast<uint2*>(codes)[b] = make_uint2(lo, hi);
     bscale[b] = uint8_t(sb);
