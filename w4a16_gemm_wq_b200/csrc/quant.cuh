@@ -229,13 +229,26 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(const uint16_t* __restr
     uint32_t lo = 0, hi = 0;
     if (d != 0.0f) {
       const float denom = __fmul_rn(d, g);
-      // the IEEE quotient, then two codes per conversion instruction
+      const float rcp = __frcp_rn(denom);
+      // Codes of the IEEE quotients w / denom, two per conversion.  t = w * rcp is
+      // within 2^-22 (relative) of the quotient; when t * (1 - 2^-19) and
+      // t * (1 + 2^-19) convert to the same pair of codes as t, every value
+      // between them does (rounding is monotonic), the quotient included.  Only
+      // pairs near a rounding boundary take the divisions.
+      uint32_t pairs[8];
 #pragma unroll
-      for (int j = 0; j < 8; j += 2)
-        lo |= e2m1x2_rn_sat(__fdiv_rn(w[j], denom), __fdiv_rn(w[j + 1], denom)) << (4 * j);
+      for (int j = 0; j < 16; j += 2) {
+        const float t0 = __fmul_rn(w[j], rcp), t1 = __fmul_rn(w[j + 1], rcp);
+        const uint32_t c = e2m1x2_rn_sat(t0, t1);
+        const uint32_t cl = e2m1x2_rn_sat(__fmul_rn(t0, 1.0f - 0x1p-19f), __fmul_rn(t1, 1.0f - 0x1p-19f));
+        const uint32_t ch = e2m1x2_rn_sat(__fmul_rn(t0, 1.0f + 0x1p-19f), __fmul_rn(t1, 1.0f + 0x1p-19f));
+        pairs[j >> 1] = (c == cl && c == ch) ? c : e2m1x2_rn_sat(__fdiv_rn(w[j], denom), __fdiv_rn(w[j + 1], denom));
+      }
 #pragma unroll
-      for (int j = 0; j < 8; j += 2)
-        hi |= e2m1x2_rn_sat(__fdiv_rn(w[8 + j], denom), __fdiv_rn(w[9 + j], denom)) << (4 * j);
+      for (int q = 0; q < 4; ++q) {
+        lo |= pairs[q] << (8 * q);
+        hi |= pairs[4 + q] << (8 * q);
+      }
     }
     reinterpret_cast<uint2*>(codes)[b] = make_uint2(lo, hi);
     bscale[b] = uint8_t(sb);
