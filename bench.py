@@ -32,6 +32,8 @@ METRIC = "W4A16 linear GB/s (M=1) and TFLOP/s (M≥512) as % of B200 roofline"
 WORKLOAD = ("decode GEMV sweep, M=1: K x N in {2048x2048, 2048x256, 2048x11008, 11008x2048} "
             "x {INT4 g128, INT4 g64, NVFP4}, bf16 activations")
 FORMATS = (("int4", 128), ("int4", 64), ("nvfp4", 0))
+# measured DRAM traffic of one grouped-GEMV launch of the sweep (ncu, same kernel build)
+TC_LAUNCH_DRAM_BYTES = 81_224_448 + 2_429_440
 
 
 def load_peaks():
@@ -349,7 +351,12 @@ def run_ours(args):
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "kernel": "gemv_tc_kernel", "achieved": round(achieved, 1),
                      "peak": peaks["hbm"], "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                     "peak_source": peaks["source"], "traffic": None},
+                     "peak_source": peaks["source"],
+                     # DRAM bytes read + written by one launch of this kernel build on this
+                     # workload, from the ncu capture summarised in profiles/ (81.22 + 2.43 MB)
+                     "traffic": TC_LAUNCH_DRAM_BYTES,
+                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
+                                       "(profiles/gemv_tc_kernel_decode_sweep_grouped.md)"},
         "e2e": {"value": round(ws * step_bytes * args.steps / (ms2 * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps,
