@@ -12,8 +12,12 @@
  *  - "quantization primer" (xingyuwang.me), section 2: asymmetric
  *    q = round(x/s) + z, x_hat = (q - z) s with clipping; section 3:
  *    per-group scales; section 4: W4A16 (4-bit weights, 16-bit
- *    activations); section 12: FP8 E4M3 bit layout; section 13: a fused
- *    kernel reads compressed weights and dequantizes inside the matmul.
+ *    activations); section 6: GPTQ (quantize, estimate the error with
+ *    second-order information, adjust the remaining weights); section 12:
+ *    FP8 E4M3 bit layout; section 13: a fused kernel reads compressed
+ *    weights and dequantizes inside the matmul.
+ *  - the ms-swift article (maplevalley.com.cn): GPTQ from 128-512
+ *    calibration samples with group size 128 and no activation reordering.
  *  - "OmniQuant" tutorial (cyqw.cn), section 2.1: scale and zero point;
  *    section 2.2.2: the equivalence Y = (X s)(W / s); section 4.2: W4A4.
  *
