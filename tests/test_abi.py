@@ -80,3 +80,44 @@ def test_binding_refuses_requantizing():
     p = wq.PackedInt4(None, None, None, 1, 32, 64, 1)
     with pytest.raises(ValueError):
         wq.wq_quantize_int4(p)
+
+
+def test_gptq_and_shared_awq_validate_on_the_host(lib):
+    P = ctypes.c_void_p
+    good = P(1 << 20)
+    bad = P((1 << 20) + 8)
+    # GPTQ: unsupported group, null W, misaligned W, zeros without / with a zero point
+    assert lib.wq_gptq_int4(good, 16, 256, good, 256, 1, good, good, good, None) == wq.WQ_ERR_UNSUPPORTED
+    assert lib.wq_gptq_int4(None, 16, 256, good, 64, 1, good, good, good, None) == wq.WQ_ERR_ARG
+    assert lib.wq_gptq_int4(bad, 16, 256, good, 64, 1, good, good, good, None) == wq.WQ_ERR_ARG
+    assert lib.wq_gptq_int4(good, 16, 256, good, 64, 1, good, good, None, None) == wq.WQ_ERR_ARG
+    assert lib.wq_gptq_int4(good, 16, 256, good, 64, 0, good, good, good, None) == wq.WQ_ERR_ARG
+    assert lib.wq_gptq_int4(good, 16, 256, None, 64, 1, good, good, good, None) == wq.WQ_ERR_ARG
+    # shared-s AWQ: no matrices, a null or misaligned one, an empty calibration set
+    ptrs = (ctypes.c_void_p * 2)(1 << 20, 1 << 21)
+    ns = (ctypes.c_int64 * 2)(16, 8)
+    args = (256, good, 4, None, good, 20, 64, good, good, good, good, 1 << 30, None)
+    assert lib.awq_search_scale_shared(ctypes.cast(ptrs, P), ctypes.cast(ns, P), 0, *args) == wq.WQ_ERR_ARG
+    nulls = (ctypes.c_void_p * 2)(1 << 20, None)
+    assert lib.awq_search_scale_shared(ctypes.cast(nulls, P), ctypes.cast(ns, P), 2, *args) == wq.WQ_ERR_ARG
+    odd = (ctypes.c_void_p * 2)(1 << 20, (1 << 21) + 8)
+    assert lib.awq_search_scale_shared(ctypes.cast(odd, P), ctypes.cast(ns, P), 2, *args) == wq.WQ_ERR_ARG
+    empty = (256, good, 0, None, good, 20, 64, good, good, good, good, 1 << 30, None)
+    assert lib.awq_search_scale_shared(ctypes.cast(ptrs, P), ctypes.cast(ns, P), 2, *empty) == wq.WQ_ERR_ARG
+
+
+def test_split_k_plan_is_host_logic():
+    # the prefill GEMM splits K only for few output tiles and long K (>= 24 k-blocks per
+    # split); the workspace query is the plan's size and 0 when nothing splits
+    split = [(512, 256, 11008), (512, 2048, 11008), (2048, 256, 4096)]
+    unsplit = [(512, 256, 2048), (8192, 11008, 2048), (2048, 2048, 2048), (16, 256, 11008)]
+    for M, N, K in split:
+        assert wq.linear_workspace_size(M, N, K, wq.WQ_FMT_INT4) > 0, (M, N, K)
+        assert wq.linear_workspace_size(M, N, K, wq.WQ_FMT_NVFP4) > 0, (M, N, K)
+    for M, N, K in unsplit:
+        assert wq.linear_workspace_size(M, N, K, wq.WQ_FMT_INT4) == 0, (M, N, K)
+    # 512 x 256 x 11008: 8 tiles of 128 x 128, 7 CTAs per tile (172 k-blocks / 24), fp32
+    # partial tiles plus one counter per tile (each part 256-byte aligned)
+    tiles, splits = 8, 7
+    part = tiles * splits * 128 * 128 * 4
+    assert wq.linear_workspace_size(512, 256, 11008, wq.WQ_FMT_INT4) == part + 256
