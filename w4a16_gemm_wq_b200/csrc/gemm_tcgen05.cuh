@@ -374,14 +374,21 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
       uint32_t sbv[4] = {0, 0, 0, 0};  // NVFP4: the k-block's 4 E4M3 block scales as bf16x2 {sb, sb}
       if (FMT == GEMM_INT4) {
         const int g = (kb * kGemmBK) >> a.log2g;
+        if (a.log2g == 5) {  // G = 32: groups g (words 0-3) and g + 1 (words 4-7)
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int gh = g + (a.log2g == 5 ? h : 0);
-          const float sc = __half2float(__ushort_as_half(uint16_t(a.log2g == 5 && h ? cur_a >> 16 : cur_a)));
-          const int z = (cur_b >> (4 * (gh & 7))) & 0xF;
-          sc2[h] = pack_bf16x2(sc, sc);
-          const uint32_t zb = 0x4300u | uint32_t(z);  // bf16(128 + z)
-          zoff2[h] = zb | (zb << 16);
+          for (int h = 0; h < 2; ++h) {
+            const float sc = __half2float(__ushort_as_half(uint16_t(h ? cur_a >> 16 : cur_a)));
+            const int z = (cur_b >> (4 * ((g + h) & 7))) & 0xF;
+            sc2[h] = pack_bf16x2(sc, sc);
+            const uint32_t zb = 0x4300u | uint32_t(z);  // bf16(128 + z)
+            zoff2[h] = zb | (zb << 16);
+          }
+        } else {  // one group covers the k-block
+          const float sc = __half2float(__ushort_as_half(uint16_t(cur_a)));
+          const int z = (cur_b >> (4 * (g & 7))) & 0xF;
+          sc2[0] = sc2[1] = pack_bf16x2(sc, sc);
+          const uint32_t zb = 0x4300u | uint32_t(z);
+          zoff2[0] = zoff2[1] = zb | (zb << 16);
         }
       } else {
 #pragma unroll
