@@ -32,8 +32,24 @@ METRIC = "W4A16 linear GB/s (M=1) and TFLOP/s (M≥512) as % of B200 roofline"
 WORKLOAD = ("decode GEMV sweep, M=1: K x N in {2048x2048, 2048x256, 2048x11008, 11008x2048} "
             "x {INT4 g128, INT4 g64, NVFP4}, bf16 activations")
 FORMATS = (("int4", 128), ("int4", 64), ("nvfp4", 0))
-# measured DRAM traffic of one grouped-GEMV launch of the sweep (ncu, same kernel build)
-TC_LAUNCH_DRAM_BYTES = 81_224_448 + 2_429_440
+# DRAM traffic of one grouped-GEMV launch of the sweep from an ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), valid only for the kernel
+# source it was taken on: the bench reports it when gemv_tc.cuh still hashes to
+# the recorded value and null otherwise.
+TC_TRAFFIC_CAPTURE = {"bytes": 81_224_448 + 2_429_440, "kernel_source_sha256_16": "322cc14da838cc97",
+                      "profile": "profiles/gemv_tc_kernel_decode_sweep_grouped.md"}
+
+
+def tc_traffic():
+    """(bytes or None, note) of the captured traffic for the current gemv_tc source."""
+    import hashlib
+    src = os.path.join(ROOT, "w4a16_gemm_wq_b200", "csrc", "gemv_tc.cuh")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    if sha == TC_TRAFFIC_CAPTURE["kernel_source_sha256_16"]:
+        return TC_TRAFFIC_CAPTURE["bytes"], ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch, "
+                                             f"kernel source {sha} ({TC_TRAFFIC_CAPTURE['profile']})")
+    return None, f"null: gemv_tc.cuh ({sha}) changed since the ncu capture ({TC_TRAFFIC_CAPTURE['kernel_source_sha256_16']})"
 
 
 def load_peaks():
@@ -338,6 +354,7 @@ def run_ours(args):
     d2h = 2 * yall.numel()
     del ggraphs, egraphs, cgraph
 
+    traffic, traffic_note = tc_traffic()
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True,
@@ -352,11 +369,8 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": "gemv_tc_kernel", "achieved": round(achieved, 1),
                      "peak": peaks["hbm"], "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
                      "peak_source": peaks["source"],
-                     # DRAM bytes read + written by one launch of this kernel build on this
-                     # workload, from the ncu capture summarised in profiles/ (81.22 + 2.43 MB)
-                     "traffic": TC_LAUNCH_DRAM_BYTES,
-                     "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
-                                       "(profiles/gemv_tc_kernel_decode_sweep_grouped.md)"},
+                     "traffic": traffic, "traffic_source": traffic_note,
+                     "algorithmic_bytes_per_launch": step_bytes},
         "e2e": {"value": round(ws * step_bytes * args.steps / (ms2 * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps,

@@ -148,10 +148,10 @@ int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scal
  * Per row, columns k = 0..K-1 in order: at a group's first column its scale
  * and zero point follow wq_quantize_int4's rule applied to the group's
  * weights as they stand; q_k as wq_quantize_int4;
- * e_k = (w_k - (q_k - z) * scale) * r_k with r_k = fp32(1 / U[k][k]); then
- * w_j = fmaf(-e_k, U[k][j], w_j)
- * for all j > k.  All in fp32, one rounding per operation, every w_j adjusted
- * in increasing k: the codes are bit-for-bit deterministic.  Returns
+ * e_k = (w_k - (q_k - z) * scale) / U[k][k]; then w_j = w_j - e_k * U[k][j]
+ * for all j > k.  All in fp32, each operation rounded on its own (no fused
+ * multiply-add), every w_j adjusted in increasing k: the codes are bit-for-bit
+ * deterministic.  Returns
  * WQ_ERR_UNSUPPORTED if one row of K fp32 weights plus a G x G tile of U does
  * not fit the GPU's shared memory (K up to ~40000). */
 int wq_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int group_size,

@@ -279,8 +279,9 @@ def gptq_hessian_factor(X, damp: float = 0.01) -> np.ndarray:
 def gptq_int4(W, U, group_size: int, zero_point: int = 1, want_err: bool = False) -> dict:
     """GPTQ INT4 pack of W [N, K] with the inverse-Hessian factor U (fp32 [K, K]):
     columns in order, group scale/zero from the weights as they stand at the
-    group's first column, error e_k = (w_k - deq(q_k)) * fp32(1 / U[k][k]), later columns
-    w_j -= e_k U[k][j] in fp32.  Returns the pack (and e [N, K] fp32)."""
+    group's first column, error e_k = (w_k - deq(q_k)) / U[k][k], later columns
+    w_j = w_j - e_k U[k][j], fp32 with every operation rounded on its own.
+    Returns the pack (and e [N, K] fp32)."""
     w = as_bits16(W)
     N, K = w.shape
     u = np.ascontiguousarray(U, dtype=np.float32)

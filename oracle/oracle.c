@@ -437,12 +437,12 @@ int oracle_awq_search(const uint16_t* W, int64_t N, int64_t K, const uint16_t* X
  *  - a group's scale and zero point come from the plain quantizer's min-max
  *    rule applied to the group's weights as they stand when its first column
  *    is reached (after the adjustments from earlier columns);
- *  - the error of column k is e_k = (w_k - dequant(q_k)) * r_k, with r_k the
- *    fp32 reciprocal of U[k][k] (the division by the diagonal evaluated as one
- *    rounded reciprocal and one rounded product), and the adjustment of every
- *    later column j is w_j = fmaf(-e_k, U[k][j], w_j), in fp32 (the precision
- *    the GPU kernel takes the same decisions in), one rounding per operation,
- *    k in increasing order.
+ *  - the error of column k is e_k = (w_k - dequant(q_k)) / U[k][k], and every
+ *    later column j is adjusted by w_j = w_j - e_k * U[k][j], k in increasing
+ *    order; the arithmetic is fp32 (the precision in which the codes, an
+ *    integer decision, are taken), each +, -, *, / rounded on its own (IEEE
+ *    round-to-nearest-even; this file is compiled without contraction into
+ *    fused multiply-adds).
  * In exact arithmetic this gives W - dequant(Q) = E U row by row, which the
  * tests check.  err (optional, fp32 [N, K]) receives the e_k. */
 int oracle_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int group_size, int zero_point,
@@ -487,11 +487,10 @@ int oracle_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, in
       qweight[n * (K / 8) + k / 8] |= (uint32_t)q << (4 * (k % 8));
       /* estimate its error, scaled by the second-order information */
       const float deq = (q - z) * sc; /* exact: |q - z| <= 15, sc has 11 significant bits */
-      const float rk = 1.0f / U[k * K + k];
-      const float e = (w[k] - deq) * rk;
+      const float e = (w[k] - deq) / U[k * K + k];
       if (err) err[n * K + k] = e;
       /* adjust the weights not yet quantized */
-      for (int64_t j = k + 1; j < K; ++j) w[j] = fmaf(-e, U[k * K + j], w[j]);
+      for (int64_t j = k + 1; j < K; ++j) w[j] = w[j] - e * U[k * K + j];
     }
     free(w);
   }

@@ -57,6 +57,20 @@ def test_ragged_k_and_n(lib, K, N):
         assert_linear_close(Y, _ref_int4(p, X, inv_s), what=f"int4 {K}x{N}")
 
 
+@pytest.mark.parametrize("K", [96, 1056])
+@pytest.mark.parametrize("zp", [1, 0])
+def test_int4_g32_odd_group_count(lib, K, zp):
+    # G = 32 with an odd number of groups (K % 64 == 32): the dequantizer's last
+    # 64-wide k-block holds one real group, its upper half lies past K
+    M, N = 160, 200
+    W = synth.weight(N, K, seed=K + zp)
+    X = synth.activations(M, K, seed=K + 1)
+    inv_s = synth.act_mean_lognormal(K, seed=K).numpy().astype(np.float32)
+    p = lib.wq_quantize_int4(W.cuda(), 32, zp)
+    Y = lib.wq_linear_int4(X.cuda(), p, act_inv_s=torch.tensor(inv_s).cuda())
+    assert_linear_close(Y, _ref_int4(p, X, inv_s), what=f"int4 g32 zp={zp} K={K}")
+
+
 def _sampled_rows(M, n=24):
     rows = set(range(0, M, max(1, M // n)))
     rows.update({0, 127, 128, M - 1})

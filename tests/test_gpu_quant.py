@@ -105,3 +105,16 @@ def test_ragged_row_counts_and_long_k(lib):
     _check_nvfp4(lib, W)
     W = synth.weight(3, 32 * 3, seed=8)  # K = 96: only with G... K % 64 != 0 -> nvfp4 only
     _check_nvfp4(lib, W)
+
+
+def test_nvfp4_tiny_tensor_without_finite_reciprocal(lib):
+    # a tensor with amax ~2e-36: g and many block denominators e4m3(sb) * g fall
+    # below 2^-128, where 1 / denominator overflows fp32; the codes must still be
+    # those of the IEEE quotients w / denominator
+    W = synth.weight(8, 256, seed=9).float()
+    mag = (10.0 ** -np.repeat(np.arange(16) % 4, 16)).astype(np.float32)
+    Wt = (W * torch.tensor(mag)[None, :] * 3e-35).to(torch.bfloat16)
+    ref = oracle.quantize_nvfp4(Wt)
+    denom = oracle.e4m3_decode(ref["bscale"]).astype(np.float32) * np.float32(ref["g"])
+    assert np.any((denom > 0) & (denom < np.float32(2.0 ** -128)))
+    _check_nvfp4(lib, Wt)

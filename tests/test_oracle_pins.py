@@ -442,6 +442,28 @@ def test_gptq_identity_factor_is_plain_rtn(zp):
     np.testing.assert_array_equal(g["err"], (W.float().numpy() - oracle.dequant_int4(r)).astype(np.float32))
 
 
+@pytest.mark.parametrize("zp", [1, 0])
+def test_gptq_diagonal_factor_divides_by_the_diagonal(zp):
+    # U diagonal: the columns do not couple, so no weight is adjusted and the codes are
+    # the plain quantizer's, while each error is the IEEE fp32 quotient
+    # (w_k - deq(q_k)) / U[k][k] ("quantization primer" section 6: the error is scaled by
+    # the second-order information).  Diagonal values that are not powers of two make a
+    # reciprocal-then-multiply evaluation differ from the quotient on many elements, so
+    # that reading would fail here.
+    N, K, G = 16, 256, 64
+    W = synth.weight(N, K, seed=63, outlier_frac=0.02)
+    d = np.array([3.0, 7.0, 0.3, 1.7, 5.9, 0.11, 2.6, 9.3], dtype=np.float32)[np.arange(K) % 8]
+    g = oracle.gptq_int4(W, np.diag(d).astype(np.float32), G, zp, want_err=True)
+    r = oracle.quantize_int4(W, G, zp)
+    for key in ("qweight", "scales", "zeros"):
+        if r[key] is not None:
+            np.testing.assert_array_equal(g[key], r[key])
+    diff = W.float().numpy() - oracle.dequant_int4(r).astype(np.float32)  # fp32 - fp32, IEEE
+    quotient = diff / d[None, :]
+    np.testing.assert_array_equal(g["err"], quotient)
+    assert np.any(diff * (np.float32(1.0) / d)[None, :] != quotient)
+
+
 @pytest.mark.parametrize("G", [64, 128])
 def test_gptq_error_identity(G):
     # The adjustments accumulate so that w - deq(q) = e U for every row (U upper

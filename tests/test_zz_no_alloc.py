@@ -4,11 +4,13 @@ Some callers cannot allocate device memory at the moment they call the
 library -- a runtime that plans every device buffer up front, or code
 running where no allocator is reachable -- so they cannot pass a workspace.
 wq_linear_nvfp4_w4a4_noalloc keeps the activation pack in a fixed scratch
-array inside the library instead.  This file checks it through the C ABI
-against the workspace-taking entry point (wq_linear_nvfp4 with act_fp4 = 1),
-twice in a row (the array keeps the previous call's bytes), and that
-problems larger than the array are refused.  It is named so that pytest
-collects it last.
+array inside the library instead.  This file checks it through the C ABI,
+twice in a row (the array keeps the previous call's bytes): its output must
+be bit-identical to the workspace-taking entry point (wq_linear_nvfp4 with
+act_fp4 = 1 runs the same kernels on the same bytes), and both must match the
+oracle's fp64 product of the NVFP4-quantized activations and weights.  It
+also checks that problems larger than the array are refused.  It is named so
+that pytest collects it last.
 """
 import ctypes
 
@@ -16,9 +18,10 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import w4a16_gemm_wq_b200 as wq
 from w4a16_gemm_wq_b200 import synth
-from tests._parity import assert_linear_close
+from tests._parity import assert_linear_close, bits
 
 pytestmark = pytest.mark.gpu
 
@@ -30,6 +33,13 @@ def _noalloc(lib, X, p, Y, inv_s=None):
                                           None if inv_s is None else P(inv_s.data_ptr()), P(Y.data_ptr()),
                                           P(torch.cuda.current_stream().cuda_stream))
     return rc
+
+
+def _oracle_w4a4(X, inv_s, p):
+    xq = oracle.quantize_nvfp4(X.cpu(), s=None if inv_s is None else inv_s.cpu().numpy())
+    wh = oracle.dequant_nvfp4(dict(codes=p.codes.cpu().numpy(), bscale=p.bscale.cpu().numpy(),
+                                   g=p.global_scale.cpu().numpy()[0], N=p.N, K=p.K))
+    return oracle.matmul_abT(oracle.dequant_nvfp4(xq), wh)
 
 
 def test_noalloc_matches_workspace_entry_point_twice():
@@ -44,7 +54,8 @@ def test_noalloc_matches_workspace_entry_point_twice():
         Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         assert _noalloc(lib, X, p, Y, inv_s) == wq.WQ_OK, lib.wq_last_error().decode()
         torch.cuda.synchronize()
-        assert_linear_close(Y, ref.double().cpu().numpy(), what=f"noalloc M={M} K={K} N={N}")
+        np.testing.assert_array_equal(bits(Y), bits(ref), err_msg=f"noalloc M={M} K={K} N={N}")
+        assert_linear_close(Y, _oracle_w4a4(X, inv_s, p), what=f"noalloc vs oracle M={M} K={K} N={N}")
     assert wq.wq_device_error() == 0
 
 

@@ -9,22 +9,24 @@
 // order k = 0..K-1:
 //   k % G == 0:  the group's fp16 scale and zero point from the weights
 //                [k, k + G) as they stand now (the plain quantizer's min-max rule)
-//   q_k = quant(w_k),  e_k = (w_k - (q_k - z) sc) * r_k,  r_k = fp32 1 / U[k][k]
-//   w_j = fmaf(-e_k, U[k][j], w_j)  for every j > k
-// in fp32 with one rounding per operation.  Every w_j sees exactly the chain of
-// fmaf(-e_k, U[k][j], .) for k = 0, 1, .., j - 1 in that order, whatever the
-// schedule below, so the codes are bit-identical to the sequential definition.
+//   q_k = quant(w_k),  e_k = (w_k - (q_k - z) sc) / U[k][k]
+//   w_j = w_j - e_k U[k][j]  for every j > k
+// in fp32, every operation rounded on its own (no fused multiply-add).  Every
+// w_j sees exactly the chain of w_j - e_k U[k][j] for k = 0, 1, .., j - 1 in
+// that order, whatever the schedule below, so the codes are bit-identical to
+// the sequential definition.
 //
 // Schedule: a CTA takes R rows at a time (their working weights fp32 in shared
 // memory) and walks the K columns in blocks of G (one group each):
 //   1. the block's diagonal tile of U goes to shared memory;
 //   2. warp r runs row r's block sequentially from registers: group min/max by
-//      warp shuffles, then per column the owning lane quantizes and scales the
-//      error by r_k, the error is broadcast, and every lane adjusts its later
-//      columns of the block; the codes are packed, the scale and zero point written;
+//      warp shuffles, then per column the owning lane quantizes and divides the
+//      error by the diagonal, the error is broadcast, and every lane adjusts its
+//      later columns of the block; the codes are packed, the scale and zero point
+//      written;
 //   3. all threads apply the block's G errors to the columns after the block:
 //      thread j streams U[b..b+G)[j] (coalesced, shared by the R rows) and runs
-//      each row's fmaf chain in k order.
+//      each row's chain of adjustments in k order.
 // The sequential part is latency-bound (~G steps per block); the update part
 // is bound by reading U (K^2/2 floats per pass over R rows; L2-resident for
 // K = 2048, streamed through L2 by all CTAs together for K = 11008).
@@ -53,7 +55,7 @@ struct GptqArgs {
 
 // shared memory of one CTA: working rows, U's diagonal tile, the block's errors and codes
 __host__ __device__ inline size_t gptq_smem_bytes(int R, int64_t K, int G) {
-  return size_t(R) * size_t(K) * 4 + size_t(G) * G * 4 + size_t(R) * G * 4 + size_t(G) * 4 + size_t(R) * G;
+  return size_t(R) * size_t(K) * 4 + size_t(G) * G * 4 + size_t(R) * G * 4 + size_t(R) * G;
 }
 
 // RMAX: the largest row count of a pass this instantiation serves (4 for long
@@ -67,8 +69,7 @@ __global__ void __launch_bounds__(kGptqThreads, 1) gptq_int4_kernel(const GptqAr
   float* w = gsm;                                              // [R][K]
   float* ud = w + size_t(R) * K;                               // [G][G]
   float* errs = ud + G * G;                                    // [R][G] negated errors -e_k
-  float* dinv = errs + R * G;                                  // [G] 1 / U[k][k] of the block
-  uint8_t* qb = reinterpret_cast<uint8_t*>(dinv + G);          // [R][G]
+  uint8_t* qb = reinterpret_cast<uint8_t*>(errs + R * G);      // [R][G]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t ng = K / G, nzw = (ng + 7) / 8;
 
@@ -92,15 +93,17 @@ __global__ void __launch_bounds__(kGptqThreads, 1) gptq_int4_kernel(const GptqAr
     for (int64_t b = 0; b < K; b += G) {
       // ---- 1. U's diagonal tile
       for (int t = threadIdx.x; t < G * G; t += kGptqThreads) ud[t] = __ldg(a.U + (b + t / G) * K + b + t % G);
-      if (threadIdx.x < G) dinv[threadIdx.x] = __frcp_rn(__ldg(a.U + (b + threadIdx.x) * (K + 1)));
       __syncthreads();
 
       // ---- 2. the block, sequentially, one warp per row
       if (warp < rows) {
         constexpr int PL = G / 32;  // columns per lane
-        float v[PL];
+        float v[PL], dg[PL];  // this lane's columns and their diagonal entries U[k][k]
 #pragma unroll
-        for (int i = 0; i < PL; ++i) v[i] = w[int64_t(warp) * K + b + lane + 32 * i];
+        for (int i = 0; i < PL; ++i) {
+          v[i] = w[int64_t(warp) * K + b + lane + 32 * i];
+          dg[i] = ud[(lane + 32 * i) * (G + 1)];
+        }
         float mn = v[0], mx = v[0], amax = fabsf(v[0]);
 #pragma unroll
         for (int i = 1; i < PL; ++i) {
@@ -127,18 +130,18 @@ __global__ void __launch_bounds__(kGptqThreads, 1) gptq_int4_kernel(const GptqAr
         for (int i = 0; i < PL; ++i) {
           for (int l2 = 0; l2 < 32; ++l2) {
             const int kk = 32 * i + l2;
-            // this step's row of U's tile and the reciprocal of its diagonal, read
-            // before the step's own stores so that they leave the dependency chain
+            // this step's row of U's tile, read before the step's own stores so
+            // that the loads leave the dependency chain
             float urow[PL];
 #pragma unroll
             for (int i2 = 0; i2 < PL; ++i2) urow[i2] = ud[kk * G + lane + 32 * i2];
-            const float rk = dinv[kk];
-            // every lane quantizes its own column of slot i (no divergent branch);
-            // the lane holding column kk keeps its code and error, all take its error
+            // every lane quantizes its own column of slot i and divides its error by
+            // its own diagonal entry (no divergent branch); the lane holding column kk
+            // keeps its code and error, all take its error
             const float q = ASYM ? fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(v[i], sc)), z), 0.0f), 15.0f)
                                  : __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(v[i], sc)), -7.0f), 7.0f), 8.0f);
             const float deq = __fmul_rn(__fsub_rn(q, z), sc);  // exact: |q - z| <= 15, sc has 11 bits
-            const float e = __shfl_sync(0xFFFFFFFFu, __fmul_rn(__fsub_rn(v[i], deq), rk), l2);
+            const float e = __shfl_sync(0xFFFFFFFFu, __fdiv_rn(__fsub_rn(v[i], deq), dg[i]), l2);
             if (lane == l2) {
               qb[warp * G + kk] = uint8_t(q);
               errs[warp * G + kk] = -e;
@@ -146,7 +149,7 @@ __global__ void __launch_bounds__(kGptqThreads, 1) gptq_int4_kernel(const GptqAr
 #pragma unroll
             for (int i2 = 0; i2 < PL; ++i2) {
               const int jj = lane + 32 * i2;
-              if (jj > kk) v[i2] = __fmaf_rn(-e, urow[i2], v[i2]);
+              if (jj > kk) v[i2] = __fsub_rn(v[i2], __fmul_rn(e, urow[i2]));
             }
           }
         }
@@ -190,11 +193,13 @@ __global__ void __launch_bounds__(kGptqThreads, 1) gptq_int4_kernel(const GptqAr
 #pragma unroll
             for (int r = 0; r < RMAX; ++r)
               if (r < rows) {
+                // w - e u as w + (-e) u: negation is exact, the product and the sum
+                // each rounded (the intrinsics are never contracted into an FMA)
                 const float4 ne = *reinterpret_cast<const float4*>(errs + r * G + k0 + q);
-                acc[r] = __fmaf_rn(ne.x, u[q], acc[r]);
-                acc[r] = __fmaf_rn(ne.y, u[q + 1], acc[r]);
-                acc[r] = __fmaf_rn(ne.z, u[q + 2], acc[r]);
-                acc[r] = __fmaf_rn(ne.w, u[q + 3], acc[r]);
+                acc[r] = __fadd_rn(acc[r], __fmul_rn(ne.x, u[q]));
+                acc[r] = __fadd_rn(acc[r], __fmul_rn(ne.y, u[q + 1]));
+                acc[r] = __fadd_rn(acc[r], __fmul_rn(ne.z, u[q + 2]));
+                acc[r] = __fadd_rn(acc[r], __fmul_rn(ne.w, u[q + 3]));
               }
           }
         }

@@ -234,7 +234,10 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(const uint16_t* __restr
       // within 2^-22 (relative) of the quotient; when t * (1 - 2^-19) and
       // t * (1 + 2^-19) convert to the same pair of codes as t, every value
       // between them does (rounding is monotonic), the quotient included.  Only
-      // pairs near a rounding boundary take the divisions.
+      // pairs near a rounding boundary take the divisions.  A denominator below
+      // 2^-128 (tensors with amax under ~1e-33) has no finite reciprocal: then
+      // every pair takes the divisions.
+      const bool rcp_ok = __float_as_uint(rcp) < 0x7F800000u;
       uint32_t pairs[8];
 #pragma unroll
       for (int j = 0; j < 16; j += 2) {
@@ -242,7 +245,8 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(const uint16_t* __restr
         const uint32_t c = e2m1x2_rn_sat(t0, t1);
         const uint32_t cl = e2m1x2_rn_sat(__fmul_rn(t0, 1.0f - 0x1p-19f), __fmul_rn(t1, 1.0f - 0x1p-19f));
         const uint32_t ch = e2m1x2_rn_sat(__fmul_rn(t0, 1.0f + 0x1p-19f), __fmul_rn(t1, 1.0f + 0x1p-19f));
-        pairs[j >> 1] = (c == cl && c == ch) ? c : e2m1x2_rn_sat(__fdiv_rn(w[j], denom), __fdiv_rn(w[j + 1], denom));
+        pairs[j >> 1] = (rcp_ok && c == cl && c == ch) ? c
+                                                         : e2m1x2_rn_sat(__fdiv_rn(w[j], denom), __fdiv_rn(w[j + 1], denom));
       }
 #pragma unroll
       for (int q = 0; q < 4; ++q) {

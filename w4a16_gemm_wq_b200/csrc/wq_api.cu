@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -74,6 +75,22 @@ int check_group(int group_size, int64_t K) {
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 int launched(const char* what) { return cuda_check(cudaGetLastError(), what); }
+
+// The dynamic shared-memory limit of a kernel (cudaFuncSetAttribute) belongs
+// to the current device's context, so it is set once per device: bit d of
+// *done records device d (devices 64 and up set it on every call).  Racing
+// threads may both set it, which is harmless.
+template <typename Kern>
+int ensure_smem_attr(Kern* kern, int bytes, std::atomic<uint64_t>* done, const char* what) {
+  int dev = 0;
+  if (int e = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+  if (bit && (done->load(std::memory_order_acquire) & bit)) return WQ_OK;
+  if (int e = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes), what))
+    return e;
+  if (bit) done->fetch_or(bit, std::memory_order_acq_rel);
+  return WQ_OK;
+}
 
 // ---------------------------------------------------------------- GEMV launch
 // Launch shape of the CUDA-core GEMV, measured per weight kind on the decode
@@ -175,14 +192,10 @@ int make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int e
 template <int FMT, int BN, int BMT = wq::kGemmBM>
 int launch_gemm_prepared(const wq::GemmArgs& a, cudaStream_t st) {
   using S = wq::GemmShape<BN, BMT>;
-  static bool attr_set = false;  // per instantiation; the value is the same on every device
-  if (!attr_set) {
-    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_tcgen05_kernel<FMT, BN, BMT>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES),
-                           "gemm smem attribute"))
-      return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (int e = ensure_smem_attr(wq::gemm_tcgen05_kernel<FMT, BN, BMT>, S::SMEM_BYTES, &attr_done,
+                               "gemm smem attribute"))
+    return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((a.N + BN - 1) / BN, (a.M + BMT - 1) / BMT, a.splitk > 1 ? a.splitk : 1);
   cfg.blockDim = dim3(S::THREADS, 1, 1);
@@ -328,14 +341,10 @@ int launch_fp4_persistent(wq::Fp4Args& a, const uint8_t* wcodes, cudaStream_t st
   if (int e = make_tmap_2d(&a.tmSB, a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 16),
                            wq::kFp4PBN, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
     return e;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_fp4_persistent_kernel,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES),
-                           "fp4 persistent smem attribute"))
-      return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (int e = ensure_smem_attr(wq::gemm_fp4_persistent_kernel, S::SMEM_BYTES, &attr_done,
+                               "fp4 persistent smem attribute"))
+    return e;
   const int64_t tiles = ((a.N + wq::kFp4PBN - 1) / wq::kFp4PBN) * int64_t((a.M + wq::kGemmBM - 1) / wq::kGemmBM);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(std::min<int64_t>(tiles, 148)), 1, 1);
@@ -370,14 +379,10 @@ int launch_fp4_bn(wq::Fp4Args& a, const uint8_t* xcodes, const uint8_t* wcodes, 
       return e;
   }
   if (a.sf_tma) return launch_fp4_persistent(a, wcodes, st);
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemm_fp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                S::SMEM_BYTES),
-                           "fp4 gemm smem attribute"))
-      return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (int e = ensure_smem_attr(wq::gemm_fp4_kernel<BN>, S::SMEM_BYTES, &attr_done,
+                               "fp4 gemm smem attribute"))
+    return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((a.N + BN - 1) / BN, (a.M + wq::kGemmBM - 1) / wq::kGemmBM, 1);
   cfg.blockDim = dim3(S::THREADS, 1, 1);
@@ -579,14 +584,10 @@ bool build_tc_args(const TcCall* calls, const int* kinds, int count, int64_t M, 
 
 template <int M>
 int launch_tc_m(const wq::TcArgs& g, int nctas, size_t smem, cudaStream_t st) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (int e = cuda_check(cudaFuncSetAttribute(wq::gemv_tc_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                wq::kTcMaxSmem),
-                           "gemv_tc smem attribute"))
-      return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_done{0};
+  if (int e = ensure_smem_attr(wq::gemv_tc_kernel<M>, wq::kTcMaxSmem, &attr_done,
+                               "gemv_tc smem attribute"))
+    return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nctas, 1, 1);
   cfg.blockDim = dim3(wq::kTcThreads, 1, 1);
@@ -776,7 +777,7 @@ int wq_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int gr
     return e;
   if (int e = cuda_check(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "SM count")) return e;
   const int G = group_size;
-  const int64_t fit = (int64_t(optin) - int64_t(G) * G * 4 - int64_t(G) * 4) / (K * 4 + int64_t(G) * 5);
+  const int64_t fit = (int64_t(optin) - int64_t(G) * G * 4) / (K * 4 + int64_t(G) * 5);
   const int R = int(std::min<int64_t>({int64_t(wq::kGptqMaxRows), N, fit}));
   if (R < 1) return fail(WQ_ERR_UNSUPPORTED, "K = %lld is too long for one row in shared memory", (long long)K);
   wq::GptqArgs a = {W, U, N, K, R, qweight, scales, zeros};
