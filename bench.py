@@ -399,6 +399,10 @@ def run_ours(args):
         out["gptq"] = {"workload": "7 projections, 512 Student-t calibration tokens, INT4 G=128 asymmetric, "
                                    "columns in order",
                        "results": gptq_measure(wq, synth, torch, dev)}
+        out["whole_model"] = {"workload": "504 bf16 weight matrices ~N(0,0.02) with 0.5% outlier channels x20 "
+                                          "(36 layers x 7 projections + `_moe_gen` siblings), lognormal act-mean "
+                                          "vectors; AWQ diagonal-proxy search (20 alphas) + INT4 g64 + NVFP4 packs",
+                              "results": whole_model_measure(wq, synth, torch, dev, peaks)}
     if not args.no_prefill:
         # the FP4 library GEMMs that give the FP4 denominator run after every GPU
         # timing (their seconds at full power would slow what follows them)
@@ -569,41 +573,102 @@ def awq_measure(wq, synth, torch, dev, peaks, T=512):
 
 
 def gptq_measure(wq, synth, torch, dev, T=512, G=128):
-    """GPTQ INT4 of the 7 projections (G = 128, asymmetric, T calibration tokens).
-    The inverse-Hessian factor is prepared with PyTorch outside the timed region
-    (its time is reported apart); the timed region is the library's GPTQ kernel.
-    Work: N * K^2 / 2 fused multiply-adds of the error feedback per projection,
-    against the fp32 CUDA-core peak (148 SMs x 128 lanes x 2 flop x max SM clock)."""
-    import time
+    """GPTQ INT4 of the 7 projections (G = 128, asymmetric, T calibration tokens),
+    both library steps timed with CUDA events: the inverse-Hessian factor
+    (wq_gptq_hessian_factor, fp64) once per distinct calibration input -- q/k/v/
+    gate/up read the same normalised hidden state, o_proj and down_proj their own
+    -- and the column-by-column quantizer (wq_gptq_int4) per projection.  Work of
+    the quantizer: N * K^2 / 2 multiply-adds of error feedback per projection,
+    against the fp32 CUDA-core peak (148 SMs x 128 lanes x 2 flop x max SM clock);
+    of the factor: 2 T K^2 (Hessian) + 2/3 K^3 (Cholesky and triangular inverse)
+    fp64 flop."""
     props = torch.cuda.get_device_properties(dev)
     clock_ghz = 1.965  # max SM clock of this part
     peak = props.multi_processor_count * 128 * 2 * clock_ghz / 1e3  # TFLOP/s
-    per, tot_s, tot_flop, prep_s = {}, 0.0, 0.0, 0.0
-    for name, K, N in synth.PROJECTIONS:
-        W = synth.weight(N, K, seed=synth.layer_seed(6, K + N), device=dev)
-        X = synth.activations_student_t(T, K, seed=synth.layer_seed(6, K), device=dev)
-        torch.cuda.synchronize()
-        t0 = time.perf_counter()
-        U = wq.gptq_hessian_factor(X)
-        torch.cuda.synchronize()
-        prep_s += time.perf_counter() - t0
-        wq.wq_gptq_int4(W, U, G, 1)
+    inputs = {"q_proj": "hidden", "k_proj": "hidden", "v_proj": "hidden", "gate_proj": "hidden",
+              "up_proj": "hidden", "o_proj": "attn_out", "down_proj": "mlp_act"}
+
+    def timed_ms(fn):
+        fn()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        wq.wq_gptq_int4(W, U, G, 1)
+        fn()
         b.record()
         torch.cuda.synchronize()
-        sec = a.elapsed_time(b) * 1e-3
-        flop = float(N) * K * K  # 2 flop per fused multiply-add, K^2 / 2 of them per row
+        return a.elapsed_time(b)
+
+    factors, prep = {}, {}
+    for name, K, N in synth.PROJECTIONS:
+        src = inputs[name]
+        if src in factors:
+            continue
+        X = synth.activations_student_t(T, K, seed=synth.layer_seed(6, K + len(src)), device=dev)
+        U = torch.empty((K, K), dtype=torch.float32, device=dev)
+        ws = torch.empty(wq.gptq_factor_workspace_size(K, T), dtype=torch.uint8, device=dev)
+        ms = timed_ms(lambda: wq.wq_gptq_hessian_factor(X, out=U, ws=ws))
+        factors[src] = U
+        flop = 2.0 * T * K * K + 2.0 / 3.0 * K ** 3
+        prep[src] = {"K": K, "ms": round(ms, 3), "fp64_TFLOP/s": round(flop / (ms * 1e-3) / 1e12, 2)}
+        del ws, X
+    wq.wq_device_error()
+    per, tot_s, tot_flop = {}, 0.0, 0.0
+    for name, K, N in synth.PROJECTIONS:
+        W = synth.weight(N, K, seed=synth.layer_seed(6, K + N), device=dev)
+        U = factors[inputs[name]]
+        sec = timed_ms(lambda: wq.wq_gptq_int4(W, U, G, 1)) * 1e-3
+        flop = float(N) * K * K  # 2 flop per multiply-add, K^2 / 2 of them per row
         per[name] = {"ms": round(sec * 1e3, 3), "TFLOP/s": round(flop / sec / 1e12, 2)}
         tot_s += sec
         tot_flop += flop
-        del U, W, X
+        del W
+    prep_ms = sum(v["ms"] for v in prep.values())
+    del factors
+    torch.cuda.empty_cache()
     return {"ms_per_projection": per, "ms_total": round(tot_s * 1e3, 3),
             "TFLOP/s": round(tot_flop / tot_s / 1e12, 2), "peak_fp32_TFLOP/s": round(peak, 1),
             "frac_of_fp32_peak": round(tot_flop / tot_s / 1e12 / peak, 4), "bound": "alu",
-            "input_preparation_s": round(prep_s, 3)}
+            "factor_ms_per_input": prep, "factor_ms_total": round(prep_ms, 3),
+            "ms_total_with_factor": round(tot_s * 1e3 + prep_ms, 3)}
+
+
+def whole_model_measure(wq, synth, torch, dev, peaks):
+    """Config 5: the 504 target Linears (36 layers x 7 projections and their
+    `_moe_gen` siblings), each with its synthetic mean |activation| vector, through
+    one wq_quantize_layers call: AWQ diagonal-proxy search over 20 alphas, INT4 g64
+    pack with the chosen s, NVFP4 pack.  GB/s counts the bf16 weights read once
+    (11.098 GB) over the call's device time."""
+    import time
+    layers = synth.whole_model_layers()
+    Ws = [synth.weight(N, K, seed=sd, device=dev) for _, _, K, N, sd in layers]
+    ams = [synth.act_mean_lognormal(K, seed=sd, device=dev) for _, _, K, _, sd in layers]
+    alphas = torch.tensor(synth.ALPHA_GRID, dtype=torch.float32, device=dev)
+    prepared = wq.make_layer_items(Ws, ams, alphas.numel(), 64)
+    ws = torch.empty(max(wq.quantize_layers_workspace_size(prepared[0], alphas.numel(), 64), 16), dtype=torch.uint8,
+                     device=dev)
+    call = lambda: wq.wq_quantize_layers(None, None, alphas, 64, ws=ws, prepared=prepared)
+    call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.perf_counter()
+    a.record()
+    call()
+    b.record()
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    sec = a.elapsed_time(b) * 1e-3
+    wq.wq_device_error()
+    outs = prepared[1]
+    bf16_bytes = sum(2 * N * K for _, _, K, N, _ in layers)
+    i4 = sum(o.int4.nbytes() for o in outs)
+    nv = sum(o.nvfp4.nbytes() for o in outs)
+    res = {"matrices": len(layers), "bf16_bytes": bf16_bytes, "int4_g64_packed_bytes": i4,
+           "nvfp4_packed_bytes": nv, "ms": round(sec * 1e3, 2), "wall_ms": round(wall * 1e3, 2),
+           "GB/s": round(bf16_bytes / sec / 1e9, 1), "frac_of_hbm": round(bf16_bytes / sec / 1e9 / peaks["hbm"], 4),
+           "launches": "per matrix: AWQ proxy search, INT4 pack, NVFP4 pack (one library call for all 504)"}
+    del Ws, ams, prepared, ws, outs
+    torch.cuda.empty_cache()
+    return res
 
 
 # ---------------------------------------------------------------- oracle arm

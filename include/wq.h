@@ -142,7 +142,8 @@ int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scal
  *   W        bf16 [N, K], 16-byte aligned
  *   U        fp32 [K, K] row-major, device: the upper Cholesky factor of the
  *            damped inverse Hessian, U^T U = (2 X^T X + lambda I)^-1 over the
- *            caller's calibration tokens X (only the upper triangle is read)
+ *            caller's calibration tokens X (only the upper triangle is read),
+ *            as wq_gptq_hessian_factor computes it
  *   group_size, zero_point, qweight, scales, zeros: as wq_quantize_int4, and
  *            the same packed format (so every linear entry point takes it)
  * Per row, columns k = 0..K-1 in order: at a group's first column its scale
@@ -157,6 +158,31 @@ int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scal
 int wq_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int group_size,
                  int zero_point, uint32_t* qweight, uint16_t* scales, uint32_t* zeros,
                  void* stream);
+
+/* wq_gptq_hessian_factor -- GPTQ's second-order information from
+ * calibration tokens ("quantization primer" section 6 "GPTQ": the error of
+ * each quantized weight is estimated with approximate second-order
+ * information; the ms-swift page: it comes from 128-512 calibration samples):
+ * the factor U that wq_gptq_int4 takes,
+ *     U^T U = (H + lambda I)^-1,  H = 2 X^T X,  lambda = damp * mean(diag H),
+ * U upper triangular with a positive diagonal (unique), fp32 [K, K]
+ * row-major with zeros below the diagonal.  Computed in fp64 on the GPU:
+ * the Hessian of the bf16 tokens, the damping, a blocked Cholesky
+ * factorisation of the Hessian in reversed channel order and a blocked
+ * triangular inverse (the reversed order turns the inverse's upper factor
+ * into the inverse of an ordinary lower factor), rounded to fp32 once.
+ *   X        bf16 [T, K] calibration tokens (T > 0: an empty calibration set
+ *            is an error), 16-byte aligned
+ *   damp     relative damping (0.01 is the customary value), finite, >= 0
+ *   U        fp32 [K, K] output, 16-byte aligned
+ *   ws, ws_bytes  scratch of wq_gptq_factor_workspace_size bytes (about
+ *            16 K^2 bytes: 1.9 GB at K = 11008)
+ * K up to 65536.  A Hessian that is not positive definite (non-finite
+ * tokens, or damp = 0 with fewer independent tokens than channels) makes U
+ * NaN and is reported by the next wq_device_error as WQ_ERR_ARG. */
+int wq_gptq_factor_workspace_size(int64_t K, int64_t T, size_t* bytes);
+int wq_gptq_hessian_factor(const uint16_t* X, int64_t T, int64_t K, double damp, float* U,
+                           void* ws, size_t ws_bytes, void* stream);
 
 /* awq_search_scale -- AWQ grid search of the per-input-channel scale
  * ("Lance-Quant" section "量化应用": grid-search AWQ scale equalization;
@@ -199,6 +225,43 @@ int awq_search_scale_shared(const uint16_t* const* Ws, const int64_t* Ns, int n_
                             const uint16_t* X, int64_t T, const float* act_mean, const float* alphas,
                             int n_alpha, int group_size, float* s_out, float* loss_out, int* best_idx,
                             void* ws, size_t ws_bytes, void* stream);
+
+/* One weight matrix of wq_quantize_layers. */
+typedef struct {
+  const uint16_t* W;        /* bf16 [N, K], 16-byte aligned */
+  int64_t N, K;
+  const float* act_mean;    /* fp32 [K] mean |activation| per input channel (the
+                               calibration statistic), or NULL: no search, the INT4
+                               pack uses no scale (the plain min-max rule) */
+  float* s_out;             /* fp32 [K] chosen AWQ scale; required with act_mean */
+  float* loss_out;          /* fp32 [n_alpha] diagonal-proxy losses; required with act_mean */
+  int* best_idx;            /* int32 [1] index of the chosen alpha; required with act_mean */
+  uint32_t* qweight;        /* INT4 pack (asymmetric, group_size) of W * s, or NULL to skip */
+  uint16_t* scales;
+  uint32_t* zeros;
+  uint8_t* codes;           /* NVFP4 pack of W, or NULL to skip */
+  uint8_t* bscale;
+  float* global_scale;
+} wq_layer_item;
+
+/* wq_quantize_layers -- quantize and pack a list of Linear weights in one
+ * call, as a whole model's target layers are ("Lance-Quant", section
+ * "校准阶段": 504 target Linear layers with saved per-channel mean
+ * |activation|, min-max fallback for layers without statistics; section
+ * "量化应用": AWQ grid search then group-wise INT4 packing, and the NVFP4 pack).
+ * For each item, in order, on `stream`:
+ *   1. with act_mean: awq_search_scale with X = NULL (the diagonal-proxy loss
+ *      from the mean |activation| alone) over `alphas` at group_size;
+ *   2. with qweight: wq_quantize_int4 (asymmetric, group_size) of W with the
+ *      chosen s (no scale without act_mean);
+ *   3. with codes: wq_quantize_nvfp4 of W (no scale).
+ * Each result equals the single entry point's.  Every item is validated
+ * before anything is launched.  ws / ws_bytes: at least
+ * wq_quantize_layers_workspace_size bytes (reused item after item). */
+int wq_quantize_layers_workspace_size(const wq_layer_item* items, int count, int n_alpha,
+                                      int group_size, size_t* bytes);
+int wq_quantize_layers(const wq_layer_item* items, int count, const float* alphas, int n_alpha,
+                       int group_size, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------- stage 2: quantized Linear
  * wq_linear_int4 -- Y = (X * act_inv_s) * dequant(Wq)^T, bf16 in, fp32
@@ -296,8 +359,9 @@ int wq_selftest_timeout(int* waited_ok, void* stream);
 /* Synchronizes `stream`, then reads and clears the device error word of the
  * current GPU.  WQ_OK if no kernel reported a problem since the last call,
  * WQ_ERR_TIMEOUT if a bounded wait inside a kernel gave up (the kernel then
- * exited early and its outputs are undefined), WQ_ERR_CUDA if the stream
- * itself failed. */
+ * exited early and its outputs are undefined), WQ_ERR_ARG if
+ * wq_gptq_hessian_factor met a Hessian that is not positive definite,
+ * WQ_ERR_CUDA if the stream itself failed. */
 int wq_device_error(void* stream);
 
 #ifdef __cplusplus

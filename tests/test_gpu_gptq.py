@@ -76,12 +76,48 @@ def test_gptq_pack_runs_through_the_linears(lib):
         assert_linear_close(Y, oracle.linear(Xa, What), what=f"gptq pack M={M}")
 
 
-def test_gptq_hessian_factor_helper_matches_oracle(lib):
-    # the binding's input preparation (PyTorch fp64 linear algebra) against the oracle's
-    K = 256
-    X = synth.activations_student_t(128, K, seed=3)
-    U = wq.gptq_hessian_factor(X.cuda()).cpu().numpy()
-    np.testing.assert_allclose(U, oracle.gptq_hessian_factor(X), rtol=1e-5, atol=1e-6)
+@pytest.mark.parametrize("T,K", [(128, 256), (100, 288), (37, 1056), (512, 2048), (512, 11008)])
+def test_gptq_hessian_factor_matches_oracle(lib, T, K):
+    # the library's fp64 factor (Hessian, damping, reversed-order Cholesky, triangular
+    # inverse) against the oracle's (numpy fp64 inverse, then Cholesky), both rounded to
+    # fp32 once: K not a multiple of the 64-wide blocks (288, 1056), T not a multiple of
+    # 32, fewer tokens than channels (the damping keeps H positive definite), and the
+    # projections' K
+    X = synth.activations_student_t(T, K, seed=T + K)
+    U = lib.wq_gptq_hessian_factor(X.cuda()).cpu().numpy()
+    assert lib.wq_device_error() == 0
+    ref = oracle.gptq_hessian_factor(X)
+    assert np.all(np.tril(U, -1) == 0) and np.all(np.diag(U) > 0)
+    np.testing.assert_allclose(U, ref, rtol=1e-5, atol=1e-6 * np.abs(ref).max())
+
+
+def test_gptq_pack_with_library_factor(lib):
+    # the whole GPTQ path on the GPU (factor, then pack) against the oracle's pack with
+    # the same factor
+    K, N, T = 2048, 256, 512
+    W = synth.weight(N, K, seed=21, outlier_frac=0.005)
+    X = synth.activations_student_t(T, K, seed=22)
+    Ud = lib.wq_gptq_hessian_factor(X.cuda())
+    p = lib.wq_gptq_int4(W.cuda(), Ud, 128, 1)
+    torch.cuda.synchronize()
+    _check(p, oracle.gptq_int4(W, Ud.cpu().numpy(), 128, 1))
+
+
+def test_gptq_hessian_factor_rejects_empty_calibration(lib):
+    X = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(wq.WQError):
+        lib.wq_gptq_hessian_factor(X)
+
+
+def test_gptq_hessian_factor_reports_non_finite_tokens(lib):
+    X = synth.activations(64, 256, seed=5)
+    X[3, 17] = float("inf")
+    U = lib.wq_gptq_hessian_factor(X.cuda())
+    with pytest.raises(wq.WQError) as e:
+        lib.wq_device_error()
+    assert e.value.status == wq.WQ_ERR_ARG
+    assert torch.isnan(U).any()
+    assert lib.wq_device_error() == 0  # the word was cleared
 
 
 def test_gptq_rejects_bad_factor_shape(lib):

@@ -8,8 +8,9 @@ library's CUDA kernels.  There is no CPU fallback: if the library cannot be
 loaded every call raises.
 
 Functions carry the C names:
-    wq_quantize_int4, wq_gptq_int4, wq_quantize_nvfp4, awq_search_scale, awq_search_scale_shared,
-    wq_linear_int4, wq_linear_nvfp4, wq_linear_group, wq_device_error
+    wq_quantize_int4, wq_gptq_hessian_factor, wq_gptq_int4, wq_quantize_nvfp4, awq_search_scale,
+    awq_search_scale_shared, wq_quantize_layers, wq_linear_int4, wq_linear_nvfp4, wq_linear_group,
+    wq_device_error
 """
 from __future__ import annotations
 
@@ -37,6 +38,8 @@ SIGNATURES = {
     "awq_search_workspace_size": (_I, [_I64, _I64, _I64, _I, _I, _PSZ]),
     "wq_quantize_int4": (_I, [_P, _I64, _I64, _I, _I, _I, _P, _P, _P, _P, _P]),
     "wq_gptq_int4": (_I, [_P, _I64, _I64, _P, _I, _I, _P, _P, _P, _P]),
+    "wq_gptq_factor_workspace_size": (_I, [_I64, _I64, _PSZ]),
+    "wq_gptq_hessian_factor": (_I, [_P, _I64, _I64, ctypes.c_double, _P, _P, _SZ, _P]),
     "wq_quantize_nvfp4": (_I, [_P, _I64, _I64, _P, _P, _P, _P, _P]),
     "awq_search_scale": (_I, [_P, _I64, _I64, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P]),
     "awq_search_scale_shared": (_I, [_P, _P, _I, _I64, _P, _I64, _P, _P, _I, _I, _P, _P, _P, _P, _SZ, _P]),
@@ -44,6 +47,8 @@ SIGNATURES = {
     "wq_linear_nvfp4": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _I, _P, _P, _P, _SZ, _P]),
     "wq_linear_nvfp4_w4a4_noalloc": (_I, [_P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P]),
     "wq_linear_group": (_I, [_P, _I, _I64, _P]),
+    "wq_quantize_layers_workspace_size": (_I, [_P, _I, _I, _I, _PSZ]),
+    "wq_quantize_layers": (_I, [_P, _I, _P, _I, _I, _P, _SZ, _P]),
     "wq_selftest_timeout": (_I, [_P, _P]),
     "wq_device_error": (_I, [_P]),
 }
@@ -178,7 +183,7 @@ def wq_quantize_int4(W: torch.Tensor, group_size: int = 64, zero_point: int = 1,
 
 def wq_gptq_int4(W: torch.Tensor, U: torch.Tensor, group_size: int = 128, zero_point: int = 1) -> PackedInt4:
     """GPTQ INT4 pack of W with the inverse-Hessian factor U (fp32 [K, K] upper
-    Cholesky factor of the damped inverse Hessian; see gptq_hessian_factor).
+    Cholesky factor of the damped inverse Hessian; see wq_gptq_hessian_factor).
     Same packed format as wq_quantize_int4."""
     if isinstance(W, (PackedInt4, PackedNVFP4)):
         raise ValueError("the layer is already quantized")
@@ -197,17 +202,29 @@ def wq_gptq_int4(W: torch.Tensor, U: torch.Tensor, group_size: int = 128, zero_p
     return PackedInt4(qweight, scales, zeros, N, K, group_size, zero_point)
 
 
-def gptq_hessian_factor(X: torch.Tensor, damp: float = 0.01) -> torch.Tensor:
-    """Input preparation for wq_gptq_int4, outside the library: U (fp32 [K, K],
-    upper) with U^T U = (H + lambda I)^-1, H = 2 X^T X over calibration tokens X
-    [T, K], lambda = damp * mean(diag H).  Runs PyTorch's fp64 linear algebra
-    (matmul, Cholesky, inverse) on X's device; the quantization itself runs in
-    the library's kernel."""
-    x = X.to(torch.float64)
-    H = 2.0 * (x.T @ x)
-    H.diagonal().add_(damp * H.diagonal().mean())
-    Hinv = torch.cholesky_inverse(torch.linalg.cholesky(H))
-    return torch.linalg.cholesky(Hinv, upper=True).to(torch.float32).contiguous()
+def gptq_factor_workspace_size(K: int, T: int) -> int:
+    b = ctypes.c_size_t()
+    _check(load().wq_gptq_factor_workspace_size(K, T, ctypes.byref(b)), "wq_gptq_factor_workspace_size")
+    return b.value
+
+
+def wq_gptq_hessian_factor(X: torch.Tensor, damp: float = 0.01, out: torch.Tensor | None = None,
+                           ws: torch.Tensor | None = None) -> torch.Tensor:
+    """U (fp32 [K, K], upper) with U^T U = (2 X^T X + lambda I)^-1 for calibration
+    tokens X (bf16 [T, K]), lambda = damp * mean(diag 2 X^T X): the factor
+    wq_gptq_int4 takes, computed by the library in fp64."""
+    _dev(X, "X", torch.bfloat16)
+    if X.dim() != 2:
+        raise ValueError("X must be [T, K]")
+    T, K = X.shape
+    U = out if out is not None else torch.empty((K, K), dtype=torch.float32, device=X.device)
+    _dev(U, "out", torch.float32, (K, K))
+    need = gptq_factor_workspace_size(K, T)
+    if ws is None or ws.numel() < need:
+        ws = _workspace(need, X.device)
+    _check(load().wq_gptq_hessian_factor(_ptr(X), T, K, float(damp), _ptr(U), _ptr(ws), ws.numel(), _stream()),
+           "wq_gptq_hessian_factor")
+    return U
 
 
 def wq_quantize_nvfp4(W: torch.Tensor, scale_s=None) -> PackedNVFP4:
@@ -288,6 +305,91 @@ def awq_search_scale_shared(Ws: list, alphas: torch.Tensor, group_size: int = 64
                                        _ptr(s), _ptr(losses), _ptr(best), _ptr(ws), b.value, _stream()),
            "awq_search_scale_shared")
     return s, losses, best
+
+
+class LayerItem(ctypes.Structure):
+    """Mirror of wq_layer_item (include/wq.h)."""
+
+    _fields_ = [("W", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("act_mean", ctypes.c_void_p),
+                ("s_out", ctypes.c_void_p), ("loss_out", ctypes.c_void_p), ("best_idx", ctypes.c_void_p),
+                ("qweight", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p),
+                ("codes", ctypes.c_void_p), ("bscale", ctypes.c_void_p), ("global_scale", ctypes.c_void_p)]
+
+
+@dataclasses.dataclass
+class QuantizedLayer:
+    """Outputs of one wq_quantize_layers item (None where not requested)."""
+    int4: PackedInt4 | None
+    nvfp4: PackedNVFP4 | None
+    s: torch.Tensor | None       # fp32 [K] chosen AWQ scale
+    losses: torch.Tensor | None  # fp32 [n_alpha]
+    best: torch.Tensor | None    # int32 [1]
+
+
+def make_layer_items(Ws: list, act_means: list, n_alpha: int, group_size: int = 64, int4: bool = True,
+                     nvfp4: bool = True):
+    """(ctypes array of wq_layer_item, [QuantizedLayer]) for the weights Ws with their
+    act_mean vectors (fp32 [K] or None): the outputs are allocated here and filled by
+    every wq_quantize_layers call made with the array."""
+    if len(Ws) != len(act_means) or not Ws:
+        raise ValueError("need one act_mean (or None) per weight matrix")
+    arr = (LayerItem * len(Ws))()
+    outs = []
+    for i, (W, am) in enumerate(zip(Ws, act_means)):
+        if isinstance(W, (PackedInt4, PackedNVFP4)):
+            raise ValueError("the layer is already quantized")
+        _dev(W, f"Ws[{i}]", torch.bfloat16)
+        N, K = W.shape
+        dev = W.device
+        it = arr[i]
+        it.W, it.N, it.K = W.data_ptr(), N, K
+        s = losses = best = None
+        if am is not None:
+            _dev(am, f"act_means[{i}]", torch.float32, (K,))
+            s = torch.empty(K, dtype=torch.float32, device=dev)
+            losses = torch.empty(max(n_alpha, 4), dtype=torch.float32, device=dev)[:n_alpha]
+            best = torch.empty(4, dtype=torch.int32, device=dev)[:1]
+            it.act_mean, it.s_out = am.data_ptr(), s.data_ptr()
+            it.loss_out, it.best_idx = losses.data_ptr(), best.data_ptr()
+        p4 = pn = None
+        if int4:
+            ng = K // group_size if K % group_size == 0 else 1
+            p4 = PackedInt4(torch.empty((N, K // 8), dtype=torch.int32, device=dev),
+                            torch.empty((N, ng), dtype=torch.float16, device=dev),
+                            torch.empty((N, (ng + 7) // 8), dtype=torch.int32, device=dev), N, K, group_size, 1)
+            it.qweight, it.scales, it.zeros = p4.qweight.data_ptr(), p4.scales.data_ptr(), p4.zeros.data_ptr()
+        if nvfp4:
+            pn = PackedNVFP4(torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                             torch.empty((N, K // 16), dtype=torch.uint8, device=dev),
+                             torch.empty(4, dtype=torch.float32, device=dev)[:1], N, K)
+            it.codes, it.bscale, it.global_scale = pn.codes.data_ptr(), pn.bscale.data_ptr(), pn.global_scale.data_ptr()
+        outs.append(QuantizedLayer(p4, pn, s, losses, best))
+    return arr, outs
+
+
+def quantize_layers_workspace_size(items, n_alpha: int, group_size: int) -> int:
+    b = ctypes.c_size_t()
+    _check(load().wq_quantize_layers_workspace_size(ctypes.cast(items, ctypes.c_void_p), len(items), n_alpha,
+                                                    group_size, ctypes.byref(b)), "wq_quantize_layers_workspace_size")
+    return b.value
+
+
+def wq_quantize_layers(Ws: list, act_means: list, alphas: torch.Tensor, group_size: int = 64, int4: bool = True,
+                       nvfp4: bool = True, ws: torch.Tensor | None = None, prepared=None) -> list:
+    """Quantize and pack many Linear weights in one library call: per matrix the AWQ
+    diagonal-proxy search when its act_mean (fp32 [K] or None) is given, the INT4
+    pack with the chosen s, and the NVFP4 pack.  Returns a QuantizedLayer per matrix.
+    `prepared` = make_layer_items(...) reuses its item array and outputs."""
+    _dev(alphas, "alphas", torch.float32)
+    n_alpha = alphas.numel()
+    arr, outs = prepared if prepared is not None else make_layer_items(Ws, act_means, n_alpha, group_size, int4,
+                                                                       nvfp4)
+    need = quantize_layers_workspace_size(arr, n_alpha, group_size)
+    if ws is None or ws.numel() < need:
+        ws = _workspace(need, alphas.device)
+    _check(load().wq_quantize_layers(ctypes.cast(arr, ctypes.c_void_p), len(arr), _ptr(alphas), n_alpha, group_size,
+                                     _ptr(ws), 0 if ws is None else ws.numel(), _stream()), "wq_quantize_layers")
+    return outs
 
 
 # ---------------------------------------------------------------- stage 2

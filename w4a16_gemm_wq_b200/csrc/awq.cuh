@@ -126,6 +126,126 @@ __global__ void __launch_bounds__(kQuantThreads) awq_delta_kernel(const uint16_t
   }
 }
 
+// ------------------------------------------------------------------ diagonal proxy, all alphas at once
+// Without calibration tokens the loss of alpha_i is sum_{n,k} (a_k Delta_i[n,k])^2
+// and needs W only: one pass over W evaluates every alpha.  A CTA keeps 8 rows x
+// 1024 k of W in registers and loops over the alphas (s and 1/s per alpha from a
+// small table that stays in L2), so W is read from HBM once instead of once per
+// alpha.  The codes take the quantizer's decisions: rint(w'/scale) through a
+// reciprocal, with the IEEE division where the product lies near a rounding tie.
+// Delta = w - deq * (1/s) in fp32 and the squares are summed per thread in fp32,
+// then in fp64 across the CTA in a fixed order, one partial per (alpha, CTA).
+constexpr int kAwqProxyRows = 8;
+constexpr int kAwqProxyThreads = 128;   // 128 x 8 = 1024 k per CTA
+constexpr int kAwqProxyMaxAlphas = 32;
+
+// tab[i][k] = s = fp32(a_k ^ alpha_i), tab[n_alpha + i][k] = fp32 1 / s, tab[2 n_alpha][k] = fp32(a_k).
+__global__ void __launch_bounds__(256) awq_proxy_table_kernel(const double* __restrict__ a,
+                                                              const float* __restrict__ alphas, int n_alpha,
+                                                              int64_t K, float* __restrict__ tab) {
+  const int64_t k = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int i = blockIdx.y;
+  if (k >= K) return;
+  if (i < n_alpha) {
+    const float sv = float(pow(a[k], double(alphas[i])));
+    tab[int64_t(i) * K + k] = sv;
+    tab[int64_t(n_alpha + i) * K + k] = __frcp_rn(sv);
+  } else {
+    tab[int64_t(2 * n_alpha) * K + k] = float(a[k]);
+  }
+}
+
+// grid = (ceil(K / 1024), ceil(N / 8)); partials[i * P + p0 + blockIdx.y * gridDim.x + blockIdx.x].
+template <int G>
+__global__ void __launch_bounds__(kAwqProxyThreads) awq_proxy_kernel(const uint16_t* __restrict__ W, int64_t N,
+                                                                     int64_t K, const float* __restrict__ tab,
+                                                                     int n_alpha, double* __restrict__ partials,
+                                                                     int64_t P, int64_t p0) {
+  constexpr int LPG = G / 8;
+  __shared__ double red[kAwqProxyThreads / 32][kAwqProxyMaxAlphas];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t k = (int64_t(blockIdx.x) * kAwqProxyThreads + threadIdx.x) * 8;
+  const bool kin = k < K;
+  const int64_t row0 = int64_t(blockIdx.y) * kAwqProxyRows;
+  uint4 wr[kAwqProxyRows];
+  bool rin[kAwqProxyRows];
+#pragma unroll
+  for (int r = 0; r < kAwqProxyRows; ++r) {
+    rin[r] = kin && row0 + r < N;
+    wr[r] = rin[r] ? ldg_stream_v4(W + (row0 + r) * K + k) : make_uint4(0, 0, 0, 0);
+  }
+  float av[8];
+  if (kin) {
+    const float4 a0 = __ldg(reinterpret_cast<const float4*>(tab + int64_t(2 * n_alpha) * K + k));
+    const float4 a1 = __ldg(reinterpret_cast<const float4*>(tab + int64_t(2 * n_alpha) * K + k + 4));
+    av[0] = a0.x; av[1] = a0.y; av[2] = a0.z; av[3] = a0.w; av[4] = a1.x; av[5] = a1.y; av[6] = a1.z; av[7] = a1.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) av[j] = 0.f;
+  }
+  for (int i = 0; i < n_alpha; ++i) {
+    float sv[8], rv[8];
+    if (kin) {
+      const float* st = tab + int64_t(i) * K + k;
+      const float* rt = tab + int64_t(n_alpha + i) * K + k;
+      const float4 s0 = __ldg(reinterpret_cast<const float4*>(st)), s1 = __ldg(reinterpret_cast<const float4*>(st + 4));
+      const float4 r0 = __ldg(reinterpret_cast<const float4*>(rt)), r1 = __ldg(reinterpret_cast<const float4*>(rt + 4));
+      sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w; sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+      rv[0] = r0.x; rv[1] = r0.y; rv[2] = r0.z; rv[3] = r0.w; rv[4] = r1.x; rv[5] = r1.y; rv[6] = r1.z; rv[7] = r1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sv[j] = rv[j] = 1.f;
+    }
+    float sq = 0.f;
+#pragma unroll
+    for (int r = 0; r < kAwqProxyRows; ++r) {
+      const uint32_t u[4] = {wr[r].x, wr[r].y, wr[r].z, wr[r].w};
+      float w[8], wp[8];
+      float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        w[j] = __uint_as_float((j & 1) ? (u[j >> 1] & 0xFFFF0000u) : (u[j >> 1] << 16));
+        wp[j] = __fmul_rn(w[j], sv[j]);
+        mn = fminf(mn, wp[j]);
+        mx = fmaxf(mx, wp[j]);
+      }
+#pragma unroll
+      for (int off = 1; off < LPG; off <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      }
+      if (!rin[r]) continue;  // whole groups share rin (a group never straddles rows or K)
+      float sc;
+      group_scale_f16(__fsub_rn(mx, mn), 15.0f, &sc);
+      const float z = fminf(fmaxf(rintf(__fdiv_rn(-mn, sc)), 0.0f), 15.0f);
+      const float rsc = __frcp_rn(sc);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        // |t - wp / sc| <= ~2^-22 |t| with |t| <= ~16: rint(t) is the quotient's rint
+        // unless t lies within 1e-5 of a half-integer
+        const float t = __fmul_rn(wp[j], rsc);
+        float q = rintf(t);
+        if (fabsf(fabsf(t - truncf(t)) - 0.5f) < 1e-5f) q = rintf(__fdiv_rn(wp[j], sc));
+        q = fminf(fmaxf(__fadd_rn(q, z), 0.0f), 15.0f);
+        const float deq = __fmul_rn(__fsub_rn(q, z), sc);
+        const float v = __fmul_rn(av[j], __fsub_rn(w[j], __fmul_rn(deq, rv[j])));
+        sq = __fmaf_rn(v, v, sq);
+      }
+    }
+    double d = double(sq);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+    if (lane == 0) red[warp][i] = d;
+  }
+  __syncthreads();
+  if (int(threadIdx.x) < n_alpha) {
+    double t = 0.0;
+#pragma unroll
+    for (int w2 = 0; w2 < kAwqProxyThreads / 32; ++w2) t += red[w2][threadIdx.x];
+    partials[int64_t(threadIdx.x) * P + p0 + int64_t(blockIdx.y) * gridDim.x + blockIdx.x] = t;
+  }
+}
+
 // loss[i] = sum of partials[i*P .. i*P+P) (fp64, fixed order), best = first
 // argmin, s_out = fp32(a ^ alphas[best]).  One CTA.
 __global__ void __launch_bounds__(256) awq_finalize_kernel(const double* __restrict__ partials, int64_t P, int n_alpha,

@@ -19,6 +19,7 @@
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
 #include "gptq.cuh"
+#include "gptq_factor.cuh"
 #include "quant.cuh"
 #include "wq_common.cuh"
 
@@ -300,11 +301,20 @@ struct AwqLayout {
   int bn;
 };
 
+// Without tokens and with at most kAwqProxyMaxAlphas alphas the search runs the
+// all-alpha proxy kernel: partial slots for up to 64 stacked matrices (each
+// starts a new 8-row block), and the s / 1/s / a table in place of Delta.
+bool awq_fused_proxy(bool has_x, int n_alpha) { return !has_x && n_alpha <= wq::kAwqProxyMaxAlphas; }
+int64_t awq_proxy_kx(int64_t K) { return (K / 8 + wq::kAwqProxyThreads - 1) / wq::kAwqProxyThreads; }
+
 AwqLayout awq_layout(int64_t N, int64_t K, int64_t T, bool has_x, int n_alpha) {
   AwqLayout L = {};
   if (has_x) {
     L.bn = gemm_bn(T, N);
     L.P = ((N + L.bn - 1) / L.bn) * ((T + wq::kGemmBM - 1) / wq::kGemmBM) * (L.bn / 32);
+  } else if (awq_fused_proxy(has_x, n_alpha)) {
+    L.bn = 0;
+    L.P = awq_proxy_kx(K) * ((N + wq::kAwqProxyRows - 1) / wq::kAwqProxyRows + 63);
   } else {
     L.bn = 0;
     L.P = ((K / 8 + wq::kQuantThreads - 1) / wq::kQuantThreads) * N;
@@ -313,7 +323,12 @@ AwqLayout awq_layout(int64_t N, int64_t K, int64_t T, bool has_x, int n_alpha) {
   L.off_s = align256(L.off_a + size_t(K) * 8);
   L.off_p = align256(L.off_s + size_t(K) * 4);
   L.off_d = align256(L.off_p + size_t(n_alpha) * size_t(L.P) * 8);
-  L.total = has_x ? align256(L.off_d + size_t(N) * size_t(2 * K) * 2) : L.off_d;
+  if (has_x)
+    L.total = align256(L.off_d + size_t(N) * size_t(2 * K) * 2);
+  else if (awq_fused_proxy(has_x, n_alpha))
+    L.total = align256(L.off_d + size_t(2 * n_alpha + 1) * size_t(K) * 4);
+  else
+    L.total = L.off_d;
   return L;
 }
 
@@ -628,6 +643,62 @@ int run_tc(const TcCall* calls, const int* kinds, int count, int64_t M, cudaStre
   return WQ_OK;
 }
 
+// ---------------------------------------------------------------- GPTQ factor
+// Workspace of wq_gptq_hessian_factor: the fp64 Hessian / Cholesky factor
+// [Kp, Kp], Z [Kp, Kp], the inverses of the 64 x 64 diagonal blocks, and the
+// reversed, transposed tokens Xr [Kp, Tp] (inside Z's bytes when they fit:
+// Z is first written after the Hessian product).
+struct FacLayout {
+  int64_t Kp, Tp;
+  size_t off_a, off_z, off_dinv, off_xr, total;
+};
+
+FacLayout fac_layout(int64_t K, int64_t T) {
+  FacLayout L = {};
+  L.Kp = (K + wq::kFacB - 1) / wq::kFacB * wq::kFacB;
+  L.Tp = (T + 31) / 32 * 32;
+  const size_t mat = size_t(L.Kp) * size_t(L.Kp) * 8;
+  L.off_a = 0;
+  L.off_z = align256(mat);
+  L.off_dinv = align256(L.off_z + mat);
+  L.total = align256(L.off_dinv + size_t(L.Kp) * wq::kFacB * 8);
+  if (L.Tp <= L.Kp) {
+    L.off_xr = L.off_z;
+  } else {
+    L.off_xr = L.total;
+    L.total = align256(L.total + size_t(L.Kp) * size_t(L.Tp) * 8);
+  }
+  return L;
+}
+
+int fac_gemm(const wq::FacGemmArgs& a, bool lower, cudaStream_t st) {
+  static std::atomic<uint64_t> done_all{0}, done_lower{0};
+  const int64_t tiles = lower ? int64_t(a.mt) * (a.mt + 1) / 2 : int64_t(a.mt) * a.nt;
+  if (tiles <= 0) return WQ_OK;
+  if (lower) {
+    if (int e = ensure_smem_attr(wq::fac_gemm_nt_kernel<wq::FAC_TILES_LOWER>, wq::kFacGemmSmem, &done_lower,
+                                 "factor gemm smem attribute"))
+      return e;
+    wq::fac_gemm_nt_kernel<wq::FAC_TILES_LOWER><<<unsigned(tiles), wq::kFacThreads, wq::kFacGemmSmem, st>>>(a);
+  } else {
+    if (int e = ensure_smem_attr(wq::fac_gemm_nt_kernel<wq::FAC_TILES_ALL>, wq::kFacGemmSmem, &done_all,
+                                 "factor gemm smem attribute"))
+      return e;
+    wq::fac_gemm_nt_kernel<wq::FAC_TILES_ALL><<<unsigned(tiles), wq::kFacThreads, wq::kFacGemmSmem, st>>>(a);
+  }
+  return launched("factor gemm launch");
+}
+
+wq::FacGemmArgs fac_args(const double* A, int64_t lda, const double* B, int64_t ldb, double* C, int64_t ldc,
+                         int64_t m, int64_t n, int64_t kd, double alpha, double beta) {
+  wq::FacGemmArgs a;
+  a.A = A; a.B = B; a.C = C;
+  a.lda = lda; a.ldb = ldb; a.ldc = ldc;
+  a.mt = int(m / wq::kFacB); a.nt = int(n / wq::kFacB); a.kd = int(kd);
+  a.alpha = alpha; a.beta = beta;
+  return a;
+}
+
 // Decode GEMV up to this many activation rows, tensor-core GEMM above.
 constexpr int64_t kGemvMaxM = 16;
 
@@ -801,6 +872,98 @@ int wq_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int gr
   return zero_point ? go(wq::gptq_int4_kernel<128, true, 16>) : go(wq::gptq_int4_kernel<128, false, 16>);
 }
 
+int wq_gptq_factor_workspace_size(int64_t K, int64_t T, size_t* bytes) {
+  REQUIRE(bytes, "bytes must not be NULL");
+  if (int e = check_shape(1, K)) return e;
+  REQUIRE(K <= 65536, "K must be at most 65536 (got %lld)", (long long)K);
+  REQUIRE(T > 0 && T <= (int64_t(1) << 24), "T must be in 1..2^24 (got %lld)", (long long)T);
+  *bytes = fac_layout(K, T).total;
+  return WQ_OK;
+}
+
+int wq_gptq_hessian_factor(const uint16_t* X, int64_t T, int64_t K, double damp, float* U, void* ws,
+                           size_t ws_bytes, void* stream) {
+  if (int e = check_shape(1, K)) return e;
+  REQUIRE(K <= 65536, "K must be at most 65536 (got %lld)", (long long)K);
+  REQUIRE(T > 0, "empty calibration set: T=%lld tokens", (long long)T);
+  REQUIRE(T <= (int64_t(1) << 24), "T must be at most 2^24");
+  REQUIRE(damp >= 0.0 && damp < 1e30, "damp must be finite and non-negative");
+  REQUIRE_PTR(X);
+  REQUIRE_PTR(U);
+  const FacLayout L = fac_layout(K, T);
+  REQUIRE(ws && ws_bytes >= L.total, "workspace too small: need %zu bytes (wq_gptq_factor_workspace_size)",
+          L.total);
+  REQUIRE_PTR(ws);
+  cudaStream_t st = as_stream(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  double* A = reinterpret_cast<double*>(wsb + L.off_a);
+  double* Z = reinterpret_cast<double*>(wsb + L.off_z);
+  double* Dinv = reinterpret_cast<double*>(wsb + L.off_dinv);
+  double* Xr = reinterpret_cast<double*>(wsb + L.off_xr);
+  const int64_t Kp = L.Kp, Tp = L.Tp, B = wq::kFacB;
+
+  // 1. H' = 2 Xr Xr^T (lower tiles), damped
+  wq::fac_xr_kernel<<<dim3(unsigned(Tp / 32), unsigned(Kp / 32)), 256, 0, st>>>(X, T, K, Tp, Xr);
+  if (int e = launched("factor tokens launch")) return e;
+  if (int e = fac_gemm(fac_args(Xr, Tp, Xr, Tp, A, Kp, Kp, Kp, Tp, 2.0, 0.0), true, st)) return e;
+  wq::fac_damp_kernel<<<1, 256, 0, st>>>(A, K, Kp, damp);
+  if (int e = launched("factor damping launch")) return e;
+  // 2. blocked Cholesky of H' in place: 64-wide steps inside 256-wide super-panels;
+  // within a super-panel each step updates only the super-panel's later columns,
+  // and the rest of the trailing matrix takes one update per super-panel with a
+  // reduction depth of 256 (a quarter of the trailing-matrix traffic of
+  // updating it at every 64-wide step)
+  const int64_t SB = 4 * B;
+  for (int64_t KB = 0; KB < Kp; KB += SB) {
+    const int64_t E = std::min(KB + SB, Kp);
+    for (int64_t kb = KB; kb < E; kb += B) {
+      const int64_t e = kb + B, rest = Kp - e;
+      double* Di = Dinv + (kb / B) * B * B;
+      wq::fac_diag_kernel<<<1, 256, 0, st>>>(A, Kp, kb, Di);
+      if (int er = launched("factor diagonal block launch")) return er;
+      if (rest == 0) break;
+      double* P = A + e * Kp + kb;  // panel [rest, B]
+      if (int er = fac_gemm(fac_args(P, Kp, Di, B, P, Kp, rest, B, B, 1.0, 0.0), false, st)) return er;
+      if (e < E) {
+        if (int er = fac_gemm(fac_args(P, Kp, P, Kp, A + e * Kp + e, Kp, rest, E - e, B, -1.0, 1.0), false, st))
+          return er;
+      }
+    }
+    if (E < Kp) {
+      const double* Q = A + E * Kp + KB;  // [Kp - E, E - KB]
+      if (int er = fac_gemm(fac_args(Q, Kp, Q, Kp, A + E * Kp + E, Kp, Kp - E, Kp - E, E - KB, -1.0, 1.0), true, st))
+        return er;
+    }
+  }
+  // 3. Z = L'^-T by blocked substitution, with the same two-level blocking
+  wq::fac_eye_kernel<<<unsigned(std::min<int64_t>((Kp * Kp + 255) / 256, 148 * 16)), 256, 0, st>>>(Z, Kp);
+  if (int e = launched("factor identity launch")) return e;
+  for (int64_t KB = 0; KB < Kp; KB += SB) {
+    const int64_t E = std::min(KB + SB, Kp);
+    for (int64_t kb = KB; kb < E; kb += B) {
+      const int64_t e = kb + B;
+      const double* Di = Dinv + (kb / B) * B * B;
+      if (int er = fac_gemm(fac_args(Z + kb, Kp, Di, B, Z + kb, Kp, e, B, B, 1.0, 0.0), false, st)) return er;
+      if (e < E) {
+        if (int er = fac_gemm(fac_args(Z + kb, Kp, A + e * Kp + kb, Kp, Z + e, Kp, e, E - e, B, -1.0, 1.0), false,
+                              st))
+          return er;
+      }
+    }
+    if (E < Kp) {
+      // rows [e, E) of the super-panel's columns are still 0 (Z is upper triangular), so
+      // the update may span rows 0..E with the reduction over all its columns
+      if (int er = fac_gemm(fac_args(Z + KB, Kp, A + E * Kp + KB, Kp, Z + E, Kp, E, Kp - E, E - KB, -1.0, 1.0),
+                            false, st))
+        return er;
+    }
+  }
+  // 4. U from Z, reversed and transposed, fp32
+  const unsigned kt = unsigned((K + 31) / 32);
+  wq::fac_u_kernel<<<dim3(kt, kt), 256, 0, st>>>(Z, K, Kp, U);
+  return launched("factor output launch");
+}
+
 int wq_quantize_nvfp4(const uint16_t* W, int64_t N, int64_t K, const float* scale_s, uint8_t* codes,
                       uint8_t* bscale, float* global_scale, void* stream) {
   if (int e = check_shape(N, K)) return e;
@@ -853,6 +1016,33 @@ static int awq_search_pieces(const uint16_t* const* Ws, const int64_t* Ns, int n
 
   wq::awq_act_mean_kernel<<<unsigned((K + 255) / 256), 256, 0, st>>>(X, T, K, act_mean, a);
   if (int e = launched("awq_act_mean launch")) return e;
+  if (awq_fused_proxy(X != nullptr, n_alpha)) {
+    // one pass over each matrix for all alphas; unused partial slots stay 0
+    float* tab = reinterpret_cast<float*>(wsb + L.off_d);
+    wq::awq_proxy_table_kernel<<<dim3(unsigned((K + 255) / 256), unsigned(n_alpha + 1)), 256, 0, st>>>(
+        a, alphas, n_alpha, K, tab);
+    if (int e = launched("awq_proxy_table launch")) return e;
+    if (int e = cuda_check(cudaMemsetAsync(partials, 0, size_t(n_alpha) * size_t(L.P) * 8, st), "memset")) return e;
+    const int64_t kx = awq_proxy_kx(K);
+    int64_t p0 = 0;
+    for (int p = 0; p < n_mats; ++p) {
+      const int64_t ry = (Ns[p] + wq::kAwqProxyRows - 1) / wq::kAwqProxyRows;
+      const dim3 grid{unsigned(kx), unsigned(ry), 1u};
+      if (group_size == 32)
+        wq::awq_proxy_kernel<32><<<grid, wq::kAwqProxyThreads, 0, st>>>(Ws[p], Ns[p], K, tab, n_alpha, partials,
+                                                                        L.P, p0);
+      else if (group_size == 64)
+        wq::awq_proxy_kernel<64><<<grid, wq::kAwqProxyThreads, 0, st>>>(Ws[p], Ns[p], K, tab, n_alpha, partials,
+                                                                        L.P, p0);
+      else
+        wq::awq_proxy_kernel<128><<<grid, wq::kAwqProxyThreads, 0, st>>>(Ws[p], Ns[p], K, tab, n_alpha, partials,
+                                                                         L.P, p0);
+      if (int e = launched("awq_proxy launch")) return e;
+      p0 += kx * ry;
+    }
+    wq::awq_finalize_kernel<<<1, 256, 0, st>>>(partials, L.P, n_alpha, a, alphas, K, loss_out, best_idx, s_out);
+    return launched("awq_finalize launch");
+  }
   wq::GemmArgs g = {};
   if (X) {
     g.M = int(T); g.N = int(N); g.K = int(2 * K); g.a_kblocks = int(K / wq::kGemmBK);
@@ -906,6 +1096,76 @@ int awq_search_scale_shared(const uint16_t* const* Ws, const int64_t* Ns, int n_
                             float* s_out, float* loss_out, int* best_idx, void* ws, size_t ws_bytes, void* stream) {
   return awq_search_pieces(Ws, Ns, n_mats, K, X, T, act_mean, alphas, n_alpha, group_size, s_out, loss_out, best_idx,
                            ws, ws_bytes, stream);
+}
+
+namespace {
+int check_layer_items(const wq_layer_item* items, int count, int n_alpha, int group_size, size_t* ws_need) {
+  REQUIRE(items, "items must not be NULL");
+  REQUIRE(count > 0, "count must be positive");
+  if (int e = check_group(group_size, 128)) return e;
+  REQUIRE(n_alpha > 0 && n_alpha <= 1024, "n_alpha must be in 1..1024");
+  size_t need = 0;
+  for (int i = 0; i < count; ++i) {
+    const wq_layer_item& it = items[i];
+    if (int e = check_shape(it.N, it.K)) return e;
+    if (int e = check_group(group_size, it.K)) return e;
+    REQUIRE(it.W && aligned16(it.W), "item %d: W must be a 16-byte aligned device pointer", i);
+    if (it.act_mean) {
+      REQUIRE(aligned16(it.act_mean), "item %d: act_mean must be 16-byte aligned", i);
+      REQUIRE(it.s_out && aligned16(it.s_out), "item %d: s_out (16-byte aligned) is required with act_mean", i);
+      REQUIRE(it.loss_out && aligned16(it.loss_out), "item %d: loss_out (16-byte aligned) is required", i);
+      REQUIRE(it.best_idx && aligned16(it.best_idx), "item %d: best_idx (16-byte aligned) is required", i);
+      need = std::max(need, awq_layout(it.N, it.K, 0, false, n_alpha).total);
+    }
+    if (it.qweight) {
+      REQUIRE(aligned16(it.qweight) && it.scales && aligned16(it.scales) && it.zeros && aligned16(it.zeros),
+              "item %d: qweight, scales and zeros must be 16-byte aligned device pointers", i);
+    }
+    if (it.codes) {
+      REQUIRE(aligned16(it.codes) && it.bscale && aligned16(it.bscale) && it.global_scale &&
+                  aligned16(it.global_scale),
+              "item %d: codes, bscale and global_scale must be 16-byte aligned device pointers", i);
+    }
+  }
+  *ws_need = need;
+  return WQ_OK;
+}
+}  // namespace
+
+int wq_quantize_layers_workspace_size(const wq_layer_item* items, int count, int n_alpha, int group_size,
+                                      size_t* bytes) {
+  REQUIRE(bytes, "bytes must not be NULL");
+  return check_layer_items(items, count, n_alpha, group_size, bytes);
+}
+
+int wq_quantize_layers(const wq_layer_item* items, int count, const float* alphas, int n_alpha, int group_size,
+                       void* ws, size_t ws_bytes, void* stream) {
+  size_t need = 0;
+  if (int e = check_layer_items(items, count, n_alpha, group_size, &need)) return e;
+  if (need) {
+    REQUIRE_PTR(alphas);
+    REQUIRE(ws && ws_bytes >= need, "workspace too small: need %zu bytes (wq_quantize_layers_workspace_size)",
+            need);
+    REQUIRE_PTR(ws);
+  }
+  for (int i = 0; i < count; ++i) {
+    const wq_layer_item& it = items[i];
+    if (it.act_mean) {
+      if (int e = awq_search_pieces(&it.W, &it.N, 1, it.K, nullptr, 0, it.act_mean, alphas, n_alpha, group_size,
+                                    it.s_out, it.loss_out, it.best_idx, ws, ws_bytes, stream))
+        return e;
+    }
+    if (it.qweight) {
+      if (int e = wq_quantize_int4(it.W, it.N, it.K, 4, group_size, 1, it.act_mean ? it.s_out : nullptr, it.qweight,
+                                   it.scales, it.zeros, stream))
+        return e;
+    }
+    if (it.codes) {
+      if (int e = wq_quantize_nvfp4(it.W, it.N, it.K, nullptr, it.codes, it.bscale, it.global_scale, stream))
+        return e;
+    }
+  }
+  return WQ_OK;
 }
 
 int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* qweight,
@@ -1086,7 +1346,11 @@ int wq_device_error(void* stream) {
   if (!word) return WQ_OK;
   const unsigned zero = 0;
   if (int e = cuda_check(cudaMemcpyToSymbol(wq::g_error_word, &zero, sizeof zero), "clear error word")) return e;
-  return fail(WQ_ERR_TIMEOUT, "device error word 0x%x (1=TMA wait, 2=MMA wait, 4=pipeline wait, 8=bounds)", word);
+  if (word == wq::ERR_NOT_POSITIVE_DEFINITE)
+    return fail(WQ_ERR_ARG, "GPTQ Hessian factor: the damped Hessian is not positive definite "
+                            "(non-finite calibration tokens?); U holds NaN");
+  return fail(WQ_ERR_TIMEOUT, "device error word 0x%x (1=TMA wait, 2=MMA wait, 4=pipeline wait, 8=bounds, "
+                              "16=Hessian not positive definite)", word);
 }
 
 }  // extern "C"

@@ -103,6 +103,18 @@ def config1(seed: int = 0):
     return dict(W=w, channels=ch, X_calib=x_calib, X1=x1, X16=x16, K=K, N=N)
 
 
+def whole_model_layers():
+    """(layer, name, K, N, seed) of the 504 target Linears of the whole-model pass:
+    36 layers x (7 projections + a same-shaped `_moe_gen` sibling of each)."""
+    out = []
+    for layer in range(N_LAYERS):
+        for p, (name, K, N) in enumerate(PROJECTIONS):
+            for sib in (0, 1):
+                out.append((layer, name + ("_moe_gen" if sib else ""), K, N,
+                            layer_seed(5, LINEARS_PER_LAYER * layer + 2 * p + sib)))
+    return out
+
+
 def layer_seed(config: int, layer_index: int) -> int:
     return 1000 * config + layer_index
 
