@@ -402,7 +402,11 @@ def run_ours(args):
         out["whole_model"] = {"workload": "504 bf16 weight matrices ~N(0,0.02) with 0.5% outlier channels x20 "
                                           "(36 layers x 7 projections + `_moe_gen` siblings), lognormal act-mean "
                                           "vectors; AWQ diagonal-proxy search (20 alphas) + INT4 g64 + NVFP4 packs",
-                              "results": whole_model_measure(wq, synth, torch, dev, peaks)}
+                              "results": whole_model_measure(wq, synth, torch, dev, peaks, ws, rank, pg)}
+    if ws > 1 and not args.no_prefill:
+        out["column_parallel"] = {"workload": "gate_proj (K=2048, N=11008) INT4 g64 with its N output channels "
+                                              "split over the ranks, X replicated, one NCCL all-gather of Y",
+                                  "results": column_parallel_measure(wq, synth, torch, dev, ws, rank)}
     if not args.no_prefill:
         # the FP4 library GEMMs that give the FP4 denominator run after every GPU
         # timing (their seconds at full power would slow what follows them)
@@ -417,6 +421,7 @@ def run_ours(args):
                 r["frac_of_burst"] = round(r["TFLOP/s"] / peaks["fp4"], 4)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+        out["cpu_baselines"] = cpu_baselines()
     if pg:
         pg.barrier()
         pg.destroy_process_group()
@@ -632,14 +637,19 @@ def gptq_measure(wq, synth, torch, dev, T=512, G=128):
             "ms_total_with_factor": round(tot_s * 1e3 + prep_ms, 3)}
 
 
-def whole_model_measure(wq, synth, torch, dev, peaks):
+def whole_model_measure(wq, synth, torch, dev, peaks, world=1, rank=0, pg=None):
     """Config 5: the 504 target Linears (36 layers x 7 projections and their
     `_moe_gen` siblings), each with its synthetic mean |activation| vector, through
     one wq_quantize_layers call: AWQ diagonal-proxy search over 20 alphas, INT4 g64
     pack with the chosen s, NVFP4 pack.  GB/s counts the bf16 weights read once
-    (11.098 GB) over the call's device time."""
+    (11.098 GB) over the call's device time.  With several ranks the matrices are
+    sharded (contiguous balanced shares, no data-path collective): the time is the
+    max over ranks and the byte totals are summed."""
     import time
-    layers = synth.whole_model_layers()
+
+    from w4a16_gemm_wq_b200.dist import max_over_ranks, shard_range, sum_over_ranks
+    all_layers = synth.whole_model_layers()
+    layers = [all_layers[i] for i in shard_range(len(all_layers), world, rank)]
     Ws = [synth.weight(N, K, seed=sd, device=dev) for _, _, K, N, sd in layers]
     ams = [synth.act_mean_lognormal(K, seed=sd, device=dev) for _, _, K, _, sd in layers]
     alphas = torch.tensor(synth.ALPHA_GRID, dtype=torch.float32, device=dev)
@@ -650,24 +660,55 @@ def whole_model_measure(wq, synth, torch, dev, peaks):
     call()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
     t0 = time.perf_counter()
     a.record()
     call()
     b.record()
     torch.cuda.synchronize()
     wall = time.perf_counter() - t0
-    sec = a.elapsed_time(b) * 1e-3
+    sec, wall = max_over_ranks([a.elapsed_time(b) * 1e-3, wall], device=dev)
     wq.wq_device_error()
     outs = prepared[1]
-    bf16_bytes = sum(2 * N * K for _, _, K, N, _ in layers)
-    i4 = sum(o.int4.nbytes() for o in outs)
-    nv = sum(o.nvfp4.nbytes() for o in outs)
-    res = {"matrices": len(layers), "bf16_bytes": bf16_bytes, "int4_g64_packed_bytes": i4,
+    bf16_bytes, i4, nv = (int(v) for v in sum_over_ranks(
+        [sum(2 * N * K for _, _, K, N, _ in layers), sum(o.int4.nbytes() for o in outs),
+         sum(o.nvfp4.nbytes() for o in outs)], device=dev))
+    res = {"matrices": len(all_layers), "ranks": world, "bf16_bytes": bf16_bytes, "int4_g64_packed_bytes": i4,
            "nvfp4_packed_bytes": nv, "ms": round(sec * 1e3, 2), "wall_ms": round(wall * 1e3, 2),
            "GB/s": round(bf16_bytes / sec / 1e9, 1), "frac_of_hbm": round(bf16_bytes / sec / 1e9 / peaks["hbm"], 4),
            "launches": "per matrix: AWQ proxy search, INT4 pack, NVFP4 pack (one library call for all 504)"}
     del Ws, ams, prepared, ws, outs
     torch.cuda.empty_cache()
+    return res
+
+
+def column_parallel_measure(wq, synth, torch, dev, world, rank, reps=20):
+    """One quantized Linear split along N over the ranks (column parallel): the local
+    INT4 linear on this rank's rows of the packed weight, then one all-gather of Y.
+    Device time per call (CUDA events on the current stream, max over ranks)."""
+    from w4a16_gemm_wq_b200.dist import column_parallel_linear, max_over_ranks, shard_range, shard_rows
+    K, N = 2048, 11008
+    W = synth.weight(N, K, seed=synth.layer_seed(4, K + N), device=dev)
+    full = wq.wq_quantize_int4(W, 64, 1)
+    part = shard_rows(full, shard_range(N, world, rank))
+    del W
+    res = {}
+    for M in (1, 2048):
+        X = synth.activations(M, K, seed=synth.layer_seed(4, M), device=dev)
+        f = lambda: column_parallel_linear(X, lambda x: wq.wq_linear_int4(x, part), N, world, rank)
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            f()
+        b.record()
+        torch.cuda.synchronize()
+        us = max_over_ranks([a.elapsed_time(b) * 1e3 / reps], device=dev)[0]
+        res[f"M{M}"] = {"us": round(us, 1), "TFLOP/s": round(2.0 * M * N * K / (us * 1e-6) / 1e12, 2)}
     return res
 
 
@@ -723,6 +764,79 @@ def cpu_baseline(seconds: float = 10.0):
                       f"(fp64 dequantize + fp64 dot), {dt:.1f} s"}
 
 
+def cpu_baselines(seconds_each: float = 4.0):
+    """The oracle (plain C, fp64, OpenMP over all host cores) timed on bounded samples
+    of configs 1, 3, 4 and 5, each scaled to its config's metric and labelled
+    "extrapolated" where the sample is a part of the workload."""
+    import numpy as np
+
+    import oracle
+    from w4a16_gemm_wq_b200 import synth
+
+    cores = oracle.num_threads()
+    alphas = np.array(synth.ALPHA_GRID, dtype=np.float32)
+
+    def timed(fn):
+        fn()
+        t0, n = time.perf_counter(), 0
+        while True:
+            fn()
+            n += 1
+            dt = time.perf_counter() - t0
+            if dt >= seconds_each:
+                return dt / n, n
+
+    out = {}
+    # config 1: AWQ s from 128 calibration rows, INT4 g64 pack, Y at M = 1 and 16
+    d = synth.config1(seed=0)
+
+    def c1():
+        s_, _, _ = oracle.awq_search(d["W"], 64, np.array([0.5], dtype=np.float32), X=d["X_calib"])
+        p = oracle.quantize_int4(d["W"], 64, s=s_)
+        wh = oracle.dequant_int4(p)
+        for X in (d["X1"], d["X16"]):
+            oracle.linear(X, wh, (1.0 / s_).astype(np.float32))
+    t, n = timed(c1)
+    out["config1"] = {"value": round(t * 1e3, 3), "unit": "ms per pass", "cores": cores, "kind": "oracle",
+                      "sample": f"the whole config ({n} passes): s = mean|x|^0.5, INT4 g64 pack, Y at M = 1 and 16"}
+    # config 3: the search of k_proj (2048 x 256, T = 512, 20 alphas), scaled to the 7 projections by flops
+    W = synth.weight(256, 2048, seed=synth.layer_seed(3, 2048 + 256))
+    X = synth.activations_student_t(512, 2048, seed=synth.layer_seed(3, 2048))
+    t, n = timed(lambda: oracle.awq_search(W, 64, alphas, X=X))
+    nk = sum(N * K for _, K, N in synth.PROJECTIONS)
+    flop = 2.0 * 512 * nk * (len(alphas) + 1)
+    t7 = t * nk / (256 * 2048)
+    out["config3"] = {"value": round(t7 * 1e3, 1), "unit": "ms for the 7-projection search (extrapolated)",
+                      "GFLOP/s": round(flop / t7 / 1e9, 2), "cores": cores, "kind": "oracle",
+                      "sample": f"k_proj search at full size ({n} runs of {t:.2f} s), scaled by N*K to 7 projections"}
+    # config 4: the oracle linear on 8 rows of gate_proj (2048 x 11008, INT4 g64, dequantized weights in
+    # fp64), scaled to the 7-projection block at M = 512 / 2048 / 8192
+    Wg = synth.weight(11008, 2048, seed=synth.layer_seed(4, 2048 + 11008))
+    wh = oracle.dequant_int4(oracle.quantize_int4(Wg, 64))
+    Xr = synth.activations(8, 2048, seed=synth.layer_seed(4, 8))
+    t, n = timed(lambda: oracle.linear(Xr, wh))
+    rate = 2.0 * 8 * 11008 * 2048 / t
+    out["config4"] = {"value": round(rate / 1e9, 2), "unit": "GFLOP/s", "cores": cores, "kind": "oracle",
+                      "block_ms_extrapolated": {f"M{M}": round(2.0 * M * nk / rate * 1e3, 1) for M in (512, 2048, 8192)},
+                      "sample": f"8 rows of gate_proj in fp64 ({n} runs), the block extrapolated by flops"}
+    # config 5: proxy search + INT4 g64 pack + NVFP4 pack of q_proj, scaled to the 504 matrices by weights
+    Wq = synth.weight(2048, 2048, seed=synth.layer_seed(5, 0))
+    am = synth.act_mean_lognormal(2048, seed=synth.layer_seed(5, 0)).numpy()
+
+    def c5():
+        s_, _, _ = oracle.awq_search(Wq, 64, alphas, act_mean=am)
+        oracle.quantize_int4(Wq, 64, s=s_)
+        oracle.quantize_nvfp4(Wq)
+    t, n = timed(c5)
+    total_w = sum(N * K for _, _, K, N, _ in synth.whole_model_layers())
+    t504 = t * total_w / (2048 * 2048)
+    out["config5"] = {"value": round(2.0 * total_w / t504 / 1e9, 3), "unit": "GB/s of bf16 weights (extrapolated)",
+                      "seconds_for_504": round(t504, 1), "cores": cores, "kind": "oracle",
+                      "sample": f"q_proj: 20-alpha proxy search + INT4 g64 + NVFP4 ({n} runs of {t:.2f} s), "
+                                f"scaled by weight count to the 504 matrices"}
+    return out
+
+
 def run_reference(args):
     ws, rank, local = dist_env()
     if rank != 0:
@@ -749,6 +863,52 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_case(name: str):
+    """One small invocation of one stage-1 kernel for an ncu capture (inputs larger
+    than L2, a few GB on the device at most); prints the device error word."""
+    import torch
+
+    import w4a16_gemm_wq_b200 as wq
+    from w4a16_gemm_wq_b200 import synth
+
+    dev = torch.device("cuda")
+    wq.load()
+    if name in ("quant", "nvfp4"):
+        W = synth.weight(16384, 8192, seed=1, device=dev)  # 268 MB of bf16
+        s = synth.act_mean_lognormal(8192, seed=1, device=dev).sqrt()
+        for _ in range(2):
+            wq.wq_quantize_int4(W, 64, 1, s) if name == "quant" else wq.wq_quantize_nvfp4(W)
+    elif name == "proxy":
+        W = synth.weight(11008, 2048, seed=2, device=dev)
+        am = synth.act_mean_lognormal(2048, seed=2, device=dev)
+        wq.awq_search_scale(W, torch.tensor(synth.ALPHA_GRID, device=dev), 64, act_mean=am)
+    elif name == "awqgemm":
+        W = synth.weight(11008, 2048, seed=3, device=dev)
+        X = synth.activations_student_t(512, 2048, seed=3, device=dev)
+        wq.awq_search_scale(W, torch.tensor(synth.ALPHA_GRID[:2], device=dev), 64, X=X)
+    elif name == "gptq":
+        K, N = 11008, 512
+        W = synth.weight(N, K, seed=4, device=dev)
+        g = torch.Generator(device=dev)
+        g.manual_seed(4)
+        U = torch.triu(torch.randn(K, K, generator=g, device=dev) * 0.01, 1)
+        U.diagonal().copy_(1.0 + torch.rand(K, generator=g, device=dev))
+        wq.wq_gptq_int4(W, U, 128, 1)
+    elif name == "factor":
+        wq.wq_gptq_hessian_factor(synth.activations_student_t(512, 11008, seed=5, device=dev))
+    elif name in ("gemm_int4", "gemm_nvfp4"):
+        K, N, M = 2048, 11008, 2048
+        W = synth.weight(N, K, seed=6, device=dev)
+        X = synth.activations(M, K, seed=6, device=dev)
+        p = wq.wq_quantize_int4(W, 64, 1) if name == "gemm_int4" else wq.wq_quantize_nvfp4(W)
+        for _ in range(2):
+            wq.wq_linear_int4(X, p) if name == "gemm_int4" else wq.wq_linear_nvfp4(X, p)
+    else:
+        raise SystemExit(f"unknown case {name}")
+    torch.cuda.synchronize()
+    print(name, "ok", wq.wq_device_error())
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -759,9 +919,25 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-aux", action="store_true", help="skip the quantize and AWQ measurements")
+    ap.add_argument("--case", help="run one small kernel case for a profiler capture and exit "
+                                   "(quant, nvfp4, proxy, awqgemm, gptq, factor, gemm_int4, gemm_nvfp4)")
     args = ap.parse_args()
+    if args.case:
+        run_case(args.case)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # launch one rank per GPU on this node (the same command under torchrun)
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+               "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *sys.argv[1:]]
+        sys.exit(subprocess.call(cmd))
+    if int(os.environ.get("WORLD_SIZE", "1")) != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={os.environ.get('WORLD_SIZE')}")
     if args.impl == "reference":
         run_reference(args)
     else:

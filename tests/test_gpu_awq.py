@@ -84,7 +84,7 @@ def test_config1_awq_alpha(lib):
     _check_choice(losses_ref, best, best_ref)
 
 
-@pytest.mark.parametrize("name,K,N", [p for p in synth.PROJECTIONS if p[0] in ("q_proj", "k_proj", "gate_proj")])
+@pytest.mark.parametrize("name,K,N", synth.PROJECTIONS)
 def test_config3_full_shapes_two_alphas(lib, name, K, N):
     # full size (T = 512 calibration tokens): the GPU searches all 20 alphas; the
     # oracle's literal loss ||X Delta^T||^2 (Delta from the oracle, product in
@@ -104,6 +104,29 @@ def test_config3_full_shapes_two_alphas(lib, name, K, N):
         ref = float(np.sum(y * y))
         assert abs(losses[i] - ref) <= LOSS_RTOL * ref, (i, losses[i], ref)
     assert _ulps(s, np.power(a, float(ALPHAS[best])).astype(np.float32)) <= 4
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,K,N", [p for p in synth.PROJECTIONS if p[0] in ("q_proj", "down_proj")])
+def test_config3_full_size_search_against_oracle(lib, name, K, N):
+    # the whole config-3 search at full size (T = 512 Student-t tokens, 20 alphas, G = 64)
+    # on the oracle too (fp64 literal losses ||X Delta^T||^2): all 20 losses, the choice
+    # (equal or a near tie), s, and the pack with the chosen s bit-exact.  Minutes of
+    # fp64 on the host for down_proj.
+    T = 512
+    W = synth.weight(N, K, seed=synth.layer_seed(3, K + N))
+    X = synth.activations_student_t(T, K, seed=synth.layer_seed(3, K))
+    s, losses, best = _run(lib, W, 64, X=X)
+    s_ref, losses_ref, best_ref = oracle.awq_search(W, 64, ALPHAS, X=X)
+    np.testing.assert_allclose(losses, losses_ref, rtol=LOSS_RTOL)
+    _check_choice(losses_ref, best, best_ref)
+    a = oracle.awq_mean_abs(X)
+    assert _ulps(s, np.power(a, float(ALPHAS[best])).astype(np.float32)) <= 4
+    p = lib.wq_quantize_int4(W.cuda(), 64, 1, torch.tensor(s).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.quantize_int4(W, 64, s=s)
+    for key in ("qweight", "scales", "zeros"):
+        np.testing.assert_array_equal(bits(getattr(p, key)), ref[key])
 
 
 @pytest.mark.parametrize("G", [64, 128])

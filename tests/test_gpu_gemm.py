@@ -77,10 +77,13 @@ def _sampled_rows(M, n=24):
     return np.array(sorted(r for r in rows if r < M))
 
 
-@pytest.mark.parametrize("name,K,N", [p for p in synth.PROJECTIONS if p[0] in ("q_proj", "k_proj", "gate_proj", "down_proj")])
-@pytest.mark.parametrize("M", [512, 2048])
+@pytest.mark.parametrize("name,K,N", synth.PROJECTIONS)
+@pytest.mark.parametrize("M", [512, 2048, 8192])
 @pytest.mark.parametrize("fmt", ["int4_g64", "nvfp4"])
 def test_config4_block_projection_sampled(lib, name, K, N, M, fmt):
+    # every projection of the block at every prefill size the benchmark times, in the
+    # benchmark's launch configuration (no workspace), on sampled rows (every row band
+    # of the tiles plus the ragged tail)
     W = synth.weight(N, K, seed=synth.layer_seed(4, K + N), device="cuda")
     X = synth.activations(M, K, seed=synth.layer_seed(4, M), device="cuda")
     if fmt == "nvfp4":
@@ -92,18 +95,6 @@ def test_config4_block_projection_sampled(lib, name, K, N, M, fmt):
     rows = _sampled_rows(M)
     ref = oracle.linear(X[rows].cpu(), _deq(p))
     assert_linear_close(Y[rows], ref, what=f"{fmt} {name} M={M}")
-
-
-def test_m8192_gate_sampled(lib):
-    K, N, M = 2048, 11008, 8192
-    W = synth.weight(N, K, seed=99, device="cuda")
-    X = synth.activations(M, K, seed=98, device="cuda")
-    p = lib.wq_quantize_int4(W, 64, 1)
-    Y = lib.wq_linear_int4(X, p)
-    rows = _sampled_rows(M, 16)
-    ref = oracle.linear(X[rows].cpu(), _deq(p))
-    assert_linear_close(Y[rows], ref, what="int4 gate M=8192")
-    assert lib.wq_device_error() == 0
 
 
 @pytest.mark.parametrize("M,N", [(2300, 4200), (2300, 4100), (2300, 2100)])

@@ -247,30 +247,28 @@ __global__ void __launch_bounds__(kAwqProxyThreads) awq_proxy_kernel(const uint1
 }
 
 // loss[i] = sum of partials[i*P .. i*P+P) (fp64, fixed order), best = first
-// argmin, s_out = fp32(a ^ alphas[best]).  One CTA.
+// argmin, s_out = fp32(a ^ alphas[best]).  One CTA of 256 threads.
 __global__ void __launch_bounds__(256) awq_finalize_kernel(const double* __restrict__ partials, int64_t P, int n_alpha,
                                                            const double* __restrict__ a,
                                                            const float* __restrict__ alphas, int64_t K,
                                                            float* __restrict__ loss_out, int* __restrict__ best_out,
                                                            float* __restrict__ s_out) {
-  __shared__ double red[256];
   __shared__ double losses[1024];
   __shared__ int best_sh;
-  for (int i = 0; i < n_alpha; ++i) {
+  // one warp per alpha: lane-strided sums, then a butterfly over the lanes (a fixed
+  // order for a given P, so the losses are reproducible)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int i = warp; i < n_alpha; i += nwarps) {
     double t = 0.0;
-    for (int64_t j = threadIdx.x; j < P; j += blockDim.x) t += partials[int64_t(i) * P + j];
-    red[threadIdx.x] = t;
-    __syncthreads();
-    for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-      if (int(threadIdx.x) < w) red[threadIdx.x] += red[threadIdx.x + w];
-      __syncthreads();
+    for (int64_t j = lane; j < P; j += 32) t += partials[int64_t(i) * P + j];
+#pragma unroll
+    for (int off = 16; off; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    if (lane == 0) {
+      losses[i] = t;
+      loss_out[i] = float(t);
     }
-    if (threadIdx.x == 0) {
-      losses[i] = red[0];
-      loss_out[i] = float(red[0]);
-    }
-    __syncthreads();
   }
+  __syncthreads();
   if (threadIdx.x == 0) {
     int b = 0;
     for (int i = 1; i < n_alpha; ++i)

@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(256) fac_damp_kernel(double* H, int64_t K, int
 // into NaN, which then reaches every later entry.
 __global__ void __launch_bounds__(256) fac_diag_kernel(double* A, int64_t lda, int64_t kb, double* Dinv) {
   __shared__ double S[kFacB][kFacB + 1];
-  __shared__ double inv_piv;
+  __shared__ double col[kFacB];
   const int tid = threadIdx.x;
   double* Ab = A + kb * lda + kb;
   for (int e = tid; e < kFacB * kFacB; e += 256) {
@@ -221,31 +221,30 @@ __global__ void __launch_bounds__(256) fac_diag_kernel(double* A, int64_t lda, i
     S[i][c] = c <= i ? Ab[int64_t(i) * lda + c] : 0.0;
   }
   __syncthreads();
+  // column j: every thread derives the pivot itself (no wait on one thread), the
+  // scaled column goes to col[], then row i is updated by its 4 threads (columns
+  // c = j+1..i with c % 4 == q, independent multiply-adds)
+  const int i = tid >> 2, q = tid & 3;
   for (int j = 0; j < kFacB; ++j) {
-    if (tid == 0) {
-      const double d = S[j][j];
-      double r;
-      if (d > 0.0 && d < INFINITY) {
-        r = sqrt(d);
-      } else {
-        report_error(ERR_NOT_POSITIVE_DEFINITE);
-        r = __longlong_as_double(0x7FF8000000000000ll);  // NaN
-      }
+    const double d = S[j][j];
+    const bool ok = d > 0.0 && d < INFINITY;
+    const double r = ok ? sqrt(d) : __longlong_as_double(0x7FF8000000000000ll);  // NaN spreads to the rest
+    if (!ok && tid == 0) report_error(ERR_NOT_POSITIVE_DEFINITE);
+    const double inv = 1.0 / r;
+    if (q == 0 && i > j) col[i] = S[i][j] * inv;
+    __syncthreads();
+    if (i > j) {
+      const double li = col[i];
+      for (int c = j + 1 + ((q - j - 1) & 3); c <= i; c += 4) S[i][c] = fma(-li, col[c], S[i][c]);
+      if (q == 0) S[i][j] = li;
+    } else if (i == j && q == 0) {
       S[j][j] = r;
-      inv_piv = 1.0 / r;
-    }
-    __syncthreads();
-    if (tid > j && tid < kFacB) S[tid][j] *= inv_piv;
-    __syncthreads();
-    for (int e = tid; e < kFacB * kFacB; e += 256) {
-      const int i = e >> 6, c = e & 63;
-      if (c > j && c <= i) S[i][c] = fma(-S[i][j], S[c][j], S[i][c]);
     }
     __syncthreads();
   }
   for (int e = tid; e < kFacB * kFacB; e += 256) {
-    const int i = e >> 6, c = e & 63;
-    Ab[int64_t(i) * lda + c] = S[i][c];
+    const int ii = e >> 6, c = e & 63;
+    Ab[int64_t(ii) * lda + c] = S[ii][c];
   }
   // inverse, column by column (columns are independent): 4 lanes per column
   // split each dot product and sum it with shuffles.  Li[c][c] = 1 / L[c][c];
@@ -254,22 +253,22 @@ __global__ void __launch_bounds__(256) fac_diag_kernel(double* A, int64_t lda, i
   __shared__ double diag_inv[kFacB];
   if (tid < kFacB) diag_inv[tid] = 1.0 / S[tid][tid];
   __syncthreads();
-  const int c = tid >> 2, q = tid & 3;
+  const int c = i;  // column of this thread's group (4 lanes q per column)
   double* Li = Dinv;
-  for (int i = 0; i < kFacB; ++i) {
+  for (int row = 0; row < kFacB; ++row) {
     double v = 0.0;
-    if (i > c) {
-      for (int k = c + q; k < i; k += 4) v = fma(S[i][k], (k == c ? diag_inv[c] : S[c][k]), v);
+    if (row > c) {
+      for (int k = c + q; k < row; k += 4) v = fma(S[row][k], (k == c ? diag_inv[c] : S[c][k]), v);
     }
     v += __shfl_xor_sync(0xFFFFFFFFu, v, 1);
     v += __shfl_xor_sync(0xFFFFFFFFu, v, 2);
-    if (q == 0 && i > c) S[c][i] = -v * diag_inv[i];
+    if (q == 0 && row > c) S[c][row] = -v * diag_inv[row];
     __syncwarp();
   }
   __syncthreads();
   for (int e = tid; e < kFacB * kFacB; e += 256) {
-    const int i = e >> 6, cc = e & 63;
-    Li[e] = i < cc ? 0.0 : (i == cc ? diag_inv[i] : S[cc][i]);
+    const int rr = e >> 6, cc = e & 63;
+    Li[e] = rr < cc ? 0.0 : (rr == cc ? diag_inv[rr] : S[cc][rr]);
   }
 }
 
