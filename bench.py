@@ -330,6 +330,10 @@ def run_ours(args):
                 "us_per_step": round(pms * 1e3 / psteps, 2), "GB/s": round(ws * p_gbs, 1),
                 "roofline_frac": round(p_gbs / peaks["hbm"], 4), "launches_per_step": len(first)}
 
+    # ---- the same sweep at M = 16 (config 1's second decode size): 12 separate calls,
+    # tensor-core GEMV reading each weight once; bytes count the 16 activation and output rows
+    m16 = decode_m16_measure(wq, synth, torch, dev, sets, peaks, args.warmup, pg)
+
     # ---- end to end through the public API with host buffers (pinned), per step:
     # H2D of the step's activations (one copy), the grouped call, D2H of the 12 outputs (one copy).
     hx = xall.cpu().pin_memory()
@@ -379,6 +383,7 @@ def run_ours(args):
                                "GB/s": round(ws * step_bytes * args.steps / (ms_single * 1e-3) / 1e9, 1)},
         "per_call": per_call,
         "detail": detail,
+        "decode_m16": m16,
     }
     out["clocks"] = clk.summary()
     if not args.no_prefill:
@@ -427,6 +432,52 @@ def run_ours(args):
         pg.destroy_process_group()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def decode_m16_measure(wq, synth, torch, dev, sets, peaks, warmup, pg=None, M=16, steps=400):
+    """The decode sweep's 12 linears at M = 16 activation rows, as 12 separate calls
+    per step (weights rotating over the same copies as the M = 1 sweep), timed on the
+    device.  Bytes per step: packed weights + 2 M K activations + 2 M N outputs."""
+    from w4a16_gemm_wq_b200.dist import max_over_ranks
+    Ks = sorted({K for K, _ in synth.DECODE_SHAPES})
+    X = {K: synth.activations(M, K, seed=synth.layer_seed(2, 16 + K), device=dev) for K in Ks}
+    Y = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (_, _, _, N, _) in sets[0]]
+
+    def step(layers):
+        for j, (fmt, G, K, N, p) in enumerate(layers):
+            if fmt == "nvfp4":
+                wq.wq_linear_nvfp4(X[K], p, out=Y[j])
+            else:
+                wq.wq_linear_int4(X[K], p, out=Y[j])
+
+    for s_ in sets:
+        step(s_)
+    torch.cuda.synchronize()
+    graphs = []
+    for s_ in sets:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(s_)
+        graphs.append(g)
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    if pg:
+        pg.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    for i in range(steps):
+        graphs[i % len(graphs)].replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks([a.elapsed_time(b)], device=dev)[0]
+    nbytes = sum(p.nbytes() + 2 * M * K + 2 * M * N for (_, _, K, N, p) in sets[0])
+    gbs = nbytes * steps / (ms * 1e-3) / 1e9
+    del graphs
+    return {"how": f"the 12 linears of the decode sweep at M = {M} as 12 separate calls per step (tensor-core "
+                   "GEMV gemv_mma_kernel, weights read once), CUDA graphs rotating the weight copies",
+            "M": M, "bytes_per_step": nbytes, "us_per_step": round(ms * 1e3 / steps, 2), "GB/s": round(gbs, 1),
+            "roofline_frac": round(gbs / peaks["hbm"], 4), "launches_per_step": len(sets[0])}
 
 
 def prefill_measure(wq, synth, torch, dev, peaks, Ms=(512, 2048, 8192), reps=20, rank=0):

@@ -94,6 +94,7 @@ def test_config4_block_projection_sampled(lib, name, K, N, M, fmt):
         Y = lib.wq_linear_int4(X, p)
     rows = _sampled_rows(M)
     ref = oracle.linear(X[rows].cpu(), _deq(p))
+    assert lib.wq_device_error() == 0
     assert_linear_close(Y[rows], ref, what=f"{fmt} {name} M={M}")
 
 

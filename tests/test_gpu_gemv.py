@@ -83,3 +83,27 @@ def test_ragged_shapes_split_k(lib, K, N):
 
 def test_no_device_error_reported(lib):
     assert lib.wq_device_error() == 0
+
+
+@pytest.mark.parametrize("M", [3, 8, 9, 16])
+@pytest.mark.parametrize("K,N", [(128, 24), (2048, 2048), (2048, 300), (11008, 2048), (24576, 40)])
+@pytest.mark.parametrize("fmt", ["int4_g32", "int4_g64", "int4_g128_sym", "nvfp4"])
+def test_tensor_core_gemv_m3_to_16(lib, M, K, N, fmt):
+    # 3 <= M <= 16 with K % 128 == 0: the weights are read once and multiplied on
+    # the tensor cores (one or two n8 tiles of activation rows), split-K slices
+    # reduced through the cluster; ragged N, the projections' K, the longest K the
+    # split serves, and an act_inv_s on half the cases
+    W = synth.weight(N, K, seed=K + N + M, device="cuda")
+    X = synth.activations(M, K, seed=M + K, device="cuda")
+    inv_s = synth.act_mean_lognormal(K, seed=K).numpy().astype(np.float32) if (M + K) % 2 else None
+    s = None if inv_s is None else torch.tensor(inv_s).cuda()
+    if fmt == "nvfp4":
+        p = lib.wq_quantize_nvfp4(W)
+        Y = lib.wq_linear_nvfp4(X, p, act_inv_s=s)
+        ref = _ref_nvfp4(p, X.cpu(), inv_s)
+    else:
+        G = {"int4_g32": 32, "int4_g64": 64}.get(fmt, 128)
+        p = lib.wq_quantize_int4(W, G, 0 if fmt.endswith("sym") else 1)
+        Y = lib.wq_linear_int4(X, p, act_inv_s=s)
+        ref = _ref_int4(p, X.cpu(), inv_s)
+    assert_linear_close(Y, ref, what=f"{fmt} M={M} {K}x{N}")

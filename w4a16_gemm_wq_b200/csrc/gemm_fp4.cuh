@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(Fp4Shape<BN>::THREADS, 1) gemm_fp4_kernel(cons
       umma_commit(accum);
     }
   } else if (warp >= 4) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the scales may come from the previous kernel
     const int quarter = warp & 3;
     const bool is_b = warp >= 8;
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;

@@ -41,14 +41,18 @@ constexpr int kGemmBK = 64;
 // 128-255 of the X tile) sharing the dequantized W tile, into two tensor-
 // memory accumulators side by side (columns [0, BN) and [BN, 2 BN)), which
 // halves the dequantization per flop.
-template <int BN, int BMT = kGemmBM>
+template <int BN, int BMT = kGemmBM, bool TMA_B = false>
 struct GemmShape {
   static constexpr int STAGES = (BN == 256) ? 3 : 4;
   static constexpr int A_BYTES = BMT * kGemmBK * 2;      // bf16 X tile (16 or 32 KB)
   static constexpr int B_BYTES = BN * kGemmBK * 2;       // dequantized W tile
   static constexpr int P_BYTES = BN * kGemmBK / 2;       // packed 4-bit W tile
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
-  static constexpr int DEQ_THREADS = BN;
+  // dequantizer (then epilogue) threads: two per weight row (each 32 of a k-block's
+  // 64 k) for 128-row W tiles, so that 8 warps hide the dequantization's dependency
+  // chains; one per row for 256-row tiles; the bf16-B mode only needs the epilogue
+  static constexpr int DEQ_SPLIT = (TMA_B || BN == 256) ? 1 : 2;
+  static constexpr int DEQ_THREADS = DEQ_SPLIT * BN;
   static constexpr int THREADS = 128 + DEQ_THREADS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
@@ -227,9 +231,9 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 }
 
 template <int FMT, int BN, int BMT = kGemmBM>
-__global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
+__global__ void __launch_bounds__(GemmShape<BN, BMT, FMT == GEMM_BF16_SQ>::THREADS, 1)
     gemm_tcgen05_kernel(const __grid_constant__ GemmArgs a) {
-  using S = GemmShape<BN, BMT>;
+  using S = GemmShape<BN, BMT, FMT == GEMM_BF16_SQ>;
   static_assert(FMT != GEMM_BF16_SQ || BMT == kGemmBM, "the sum-of-squares epilogue uses one accumulator");
   constexpr int STAGES = S::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -281,7 +285,9 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_acc = *tmem_slot;
 
-  // Weights and metadata do not depend on the previous kernel; X does.
+  // Let the next kernel in the stream launch; every thread that reads global
+  // memory waits for the previous kernel first (griddepcontrol.wait is what makes
+  // its writes visible: the weights themselves may have just been quantized).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0) {
@@ -335,7 +341,10 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
     }
   } else if (warp >= DEQ_WARP0) {
     // ---------------------------------------------------------- dequantize, then epilogue
-    const int t = threadIdx.x - DEQ_WARP0 * 32;  // weight row within the tile
+    constexpr int NW = 8 / S::DEQ_SPLIT;         // packed words (8 k each) per thread and k-block
+    const int dt = threadIdx.x - DEQ_WARP0 * 32;
+    const int t = dt % BN;                       // weight row within the tile
+    const int h = dt / BN;                       // which part of the k-block (words NW h .. NW h + NW - 1)
     const int n = min(n0 + t, a.N - 1);          // rows past N dequantize row N-1 (outputs masked)
     const int ng = a.K >> a.log2g;
     const uint32_t zw_stride = (ng + 7) >> 3;
@@ -364,6 +373,7 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
         }
       }
     };
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     uint32_t meta_a, meta_b;
     fetch_meta(kbeg, meta_a, meta_b);
     for (int i = 0; i < (FMT == GEMM_BF16_SQ ? 0 : nkb); ++i) {
@@ -402,14 +412,23 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT>::THREADS, 1)
         }
       }
       if (!mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag)) { ok = false; break; }
-      const uint32_t prow = smem_u32(p_ptr(s)) + uint32_t(t * 32);
-      const uint4 q0 = ld_shared_v4(prow), q1 = ld_shared_v4(prow + 16);
-      const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      const uint32_t prow = smem_u32(p_ptr(s)) + uint32_t(t * 32 + h * NW * 4);
+      uint32_t words[NW];
+#pragma unroll
+      for (int q = 0; q < NW / 4; ++q) {
+        const uint4 qv = ld_shared_v4(prow + 16 * q);
+        words[4 * q] = qv.x; words[4 * q + 1] = qv.y; words[4 * q + 2] = qv.z; words[4 * q + 3] = qv.w;
+      }
       const uint32_t brow = b_addr(s);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint4 v = (FMT == GEMM_INT4) ? dequant_word_int4(words[j], zoff2[j >> 2], sc2[j >> 2])
-                                     : dequant_word_nvfp4(words[j], sbv[j >> 1]);
+      for (int jw = 0; jw < NW; ++jw) {
+        const int j = NW * h + jw;  // word of the k-block
+        // its scale data, selected without a runtime-indexed array
+        const bool hi4 = NW == 8 ? jw >= 4 : h != 0;            // words 4-7: second G = 32 group
+        const int blk = NW == 8 ? jw >> 1 : 2 * h + (jw >> 1);  // NVFP4 block of the word
+        const uint32_t zz = hi4 ? zoff2[1] : zoff2[0], ss = hi4 ? sc2[1] : sc2[0];
+        const uint32_t sbk = blk == 0 ? sbv[0] : blk == 1 ? sbv[1] : blk == 2 ? sbv[2] : sbv[3];
+        uint4 v = (FMT == GEMM_INT4) ? dequant_word_int4(words[jw], zz, ss) : dequant_word_nvfp4(words[jw], sbk);
         if (a.inv_s) {
           const int k = kb * kGemmBK + 8 * j;
           if (k < a.K) {

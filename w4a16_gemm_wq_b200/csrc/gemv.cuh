@@ -202,13 +202,25 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const GemvArgs a)
     }
   };
 
-  // Weights do not depend on the previous kernel in the stream: start
-  // streaming them, let the next kernel launch, and only then wait for the
-  // previous kernel's outputs (our activations) to become visible.
-  uint4 wnext[R];
-  load_w(it0, wnext);
+  // Warm L2 with this warp's first weights while the previous kernel drains (L2
+  // is the point of coherence, so a prefetch never yields stale data), let the
+  // next kernel launch, and wait for the previous kernel's writes to become
+  // visible before any load: the weights themselves may have just been written.
+  {
+    const int kb = it0 * kGemvKPerIter + lane * 32;
+    if (it0 < it1 && kb < K) {
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int n = min(n0 + r, N - 1);
+        const size_t off = FMT == FMT_INT4 ? size_t(n) * (K / 8) * 4 + size_t(kb) / 2 : size_t(n) * (K / 2) + kb / 2;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t*>(a.wq) + off));
+      }
+    }
+  }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  uint4 wnext[R];
+  load_w(it0, wnext);
 
   for (int it = it0; it < it1; ++it) {
     uint4 wv[R];

@@ -96,9 +96,15 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_int4_kernel(
   }
   if (active) {
     uint32_t word = 0;
+    // rint(w / sc) through the correctly rounded reciprocal: t = w * (1 / sc) is
+    // within 2^-23 |t| of the IEEE quotient, so its rint is the quotient's unless t
+    // lies within 2^-21 |t| of a half-integer, where the division itself is taken
+    const float rsc = __frcp_rn(sc);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float r = rintf(__fdiv_rn(w[j], sc));
+      const float t = __fmul_rn(w[j], rsc);
+      float r = rintf(t);
+      if (fabsf(fabsf(__fsub_rn(t, truncf(t))) - 0.5f) <= fabsf(t) * 0x1p-21f) r = rintf(__fdiv_rn(w[j], sc));
       const float q = ASYM ? fminf(fmaxf(__fadd_rn(r, z), 0.0f), 15.0f)
                            : __fadd_rn(fminf(fmaxf(r, -7.0f), 7.0f), 8.0f);
       word |= uint32_t(q) << (4 * j);

@@ -17,6 +17,7 @@
 #include "gemm_fp4.cuh"
 #include "gemm_tcgen05.cuh"
 #include "gemv.cuh"
+#include "gemv_mma.cuh"
 #include "gemv_tc.cuh"
 #include "gptq.cuh"
 #include "gptq_factor.cuh"
@@ -151,6 +152,57 @@ int launch_gemv(const wq::GemvArgs& a, cudaStream_t st) {
   return launch_gemv_mt<FMT, 4>(a, st);
 }
 
+// ---------------------------------------------------------------- tensor-core GEMV, 3 <= M <= 16
+// Serves K % 128 == 0 up to 8 slices of kMmaMaxSliceSteps steps (K <= 24576).
+bool gemv_mma_serves(int64_t M, int64_t K) {
+  return M >= 3 && M <= 16 && K % wq::kMmaStepK == 0 &&
+         K <= int64_t(wq::kMmaMaxSplits) * wq::kMmaMaxSliceSteps * wq::kMmaStepK;
+}
+
+template <int FMT, int NT>
+int launch_gemv_mma_nt(const wq::GemvMmaArgs& a0, cudaStream_t st) {
+  wq::GemvMmaArgs a = a0;
+  const int nsteps = a.K / wq::kMmaStepK;
+  const int gx = (a.N + wq::kMmaWarps * 16 - 1) / (wq::kMmaWarps * 16);
+  // about two CTAs per SM, at most a portable cluster of slices, each slice small
+  // enough to stage
+  int S = std::max(1, std::min({(2 * 148 + gx - 1) / gx, wq::kMmaMaxSplits, nsteps}));
+  S = std::max(S, (nsteps + wq::kMmaMaxSliceSteps - 1) / wq::kMmaMaxSliceSteps);
+  a.slice_steps = (nsteps + S - 1) / S;
+  S = (nsteps + a.slice_steps - 1) / a.slice_steps;
+  const int smem = NT * 8 * (a.slice_steps * wq::kMmaStepK * 2 + 16);
+  // the attribute is the kernel's largest staged slice, set once per device
+  constexpr int kMaxSmem = NT * 8 * (wq::kMmaMaxSliceSteps * wq::kMmaStepK * 2 + 16);
+  static std::atomic<uint64_t> attr_done{0};
+  if (int e = ensure_smem_attr(wq::gemv_mma_kernel<FMT, NT>, kMaxSmem, &attr_done, "gemv_mma smem attribute"))
+    return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(gx, S, 1);
+  cfg.blockDim = dim3(wq::kMmaWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (S > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = S;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cuda_check(cudaLaunchKernelEx(&cfg, wq::gemv_mma_kernel<FMT, NT>, a), "gemv_mma launch");
+}
+
+template <int FMT>
+int launch_gemv_mma(const wq::GemvMmaArgs& a, cudaStream_t st) {
+  return a.M <= 8 ? launch_gemv_mma_nt<FMT, 1>(a, st) : launch_gemv_mma_nt<FMT, 2>(a, st);
+}
+
 int log2i(int v) {
   int r = 0;
   while ((1 << r) < v) ++r;
@@ -192,7 +244,7 @@ int make_tmap_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int e
 // ---------------------------------------------------------------- GEMM launch
 template <int FMT, int BN, int BMT = wq::kGemmBM>
 int launch_gemm_prepared(const wq::GemmArgs& a, cudaStream_t st) {
-  using S = wq::GemmShape<BN, BMT>;
+  using S = wq::GemmShape<BN, BMT, FMT == wq::GEMM_BF16_SQ>;
   static std::atomic<uint64_t> attr_done{0};
   if (int e = ensure_smem_attr(wq::gemm_tcgen05_kernel<FMT, BN, BMT>, S::SMEM_BYTES, &attr_done,
                                "gemm smem attribute"))
@@ -1191,6 +1243,12 @@ int wq_linear_int4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uin
     g.M = int(M); g.N = int(N); g.K = int(K); g.log2g = log2i(group_size);
     return launch_gemm<wq::FMT_INT4>(g, X, qweight, as_stream(stream), ws, ws_bytes);
   }
+  if (gemv_mma_serves(M, K)) {
+    wq::GemvMmaArgs m = {};
+    m.X = X; m.inv_s = act_inv_s; m.packed = reinterpret_cast<const uint8_t*>(qweight); m.scales = scales;
+    m.zeros = zeros; m.Y = Y; m.M = int(M); m.N = int(N); m.K = int(K); m.log2g = log2i(group_size);
+    return launch_gemv_mma<wq::FMT_INT4>(m, as_stream(stream));
+  }
   wq::GemvArgs a = {};
   a.X = X; a.inv_s = act_inv_s; a.wq = qweight; a.scales = scales; a.zeros = zeros;
   a.Y = Y; a.M = int(M); a.N = int(N); a.K = int(K); a.log2g = log2i(group_size);
@@ -1230,6 +1288,12 @@ int wq_linear_nvfp4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const ui
     g.bscale = bscale; g.gscale = global_scale; g.inv_s = act_inv_s; g.Y = Y;
     g.M = int(M); g.N = int(N); g.K = int(K);
     return launch_gemm<wq::FMT_NVFP4>(g, X, codes, as_stream(stream), ws, ws_bytes);
+  }
+  if (gemv_mma_serves(M, K)) {
+    wq::GemvMmaArgs m = {};
+    m.X = X; m.inv_s = act_inv_s; m.packed = codes; m.bscale = bscale; m.gscale = global_scale;
+    m.Y = Y; m.M = int(M); m.N = int(N); m.K = int(K);
+    return launch_gemv_mma<wq::FMT_NVFP4>(m, as_stream(stream));
   }
   wq::GemvArgs a = {};
   a.X = X; a.inv_s = act_inv_s; a.wq = codes; a.bscale = bscale; a.gscale = global_scale;
