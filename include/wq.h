@@ -27,8 +27,10 @@
  *  - bf16 and fp16 values travel as their 16-bit patterns (uint16_t).
  *  - All data pointers are DEVICE pointers owned by the caller; the library
  *    allocates no memory and keeps no state except one device error word
- *    per loaded GPU (see wq_device_error) and the fixed scratch array of
- *    wq_linear_nvfp4_w4a4_noalloc.
+ *    per loaded GPU (see wq_device_error), the fixed scratch array of
+ *    wq_linear_nvfp4_w4a4_noalloc, and one internal CUDA stream per GPU that
+ *    wq_gptq_hessian_factor creates on first use (its work is joined back to
+ *    the caller's stream before the call's last launch).
  *  - `stream` is a cudaStream_t (0 = legacy default stream).  Every call is
  *    asynchronous on that stream; validation happens on the host before any
  *    launch, so an error return means nothing was launched.
@@ -179,7 +181,9 @@ int wq_gptq_int4(const uint16_t* W, int64_t N, int64_t K, const float* U, int gr
  *            16 K^2 bytes: 1.9 GB at K = 11008)
  * K up to 65536.  A Hessian that is not positive definite (non-finite
  * tokens, or damp = 0 with fewer independent tokens than channels) makes U
- * NaN and is reported by the next wq_device_error as WQ_ERR_ARG. */
+ * NaN and is reported by the next wq_device_error as WQ_ERR_ARG.  The
+ * inverse runs on an internal stream that overlaps the factorisation and
+ * joins `stream` before U is written; calls on one GPU share that stream. */
 int wq_gptq_factor_workspace_size(int64_t K, int64_t T, size_t* bytes);
 int wq_gptq_hessian_factor(const uint16_t* X, int64_t T, int64_t K, double damp, float* U,
                            void* ws, size_t ws_bytes, void* stream);

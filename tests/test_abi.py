@@ -107,17 +107,18 @@ def test_gptq_and_shared_awq_validate_on_the_host(lib):
 
 
 def test_split_k_plan_is_host_logic():
-    # the prefill GEMM splits K only for few output tiles and long K (>= 24 k-blocks per
-    # split); the workspace query is the plan's size and 0 when nothing splits
-    split = [(512, 256, 11008), (512, 2048, 11008), (2048, 256, 4096)]
-    unsplit = [(512, 256, 2048), (8192, 11008, 2048), (2048, 2048, 2048), (16, 256, 11008)]
+    # the prefill GEMM splits K only when its tiles cover under half of the SMs: at
+    # least 24 k-blocks per split for 37..73 tiles, at least 8 for fewer; the workspace
+    # query is the plan's size and 0 when nothing splits
+    split = [(512, 256, 11008), (512, 2048, 11008), (2048, 256, 4096), (512, 256, 2048)]
+    unsplit = [(512, 2048, 2048), (8192, 11008, 2048), (2048, 2048, 2048), (16, 256, 11008)]
     for M, N, K in split:
         assert wq.linear_workspace_size(M, N, K, wq.WQ_FMT_INT4) > 0, (M, N, K)
         assert wq.linear_workspace_size(M, N, K, wq.WQ_FMT_NVFP4) > 0, (M, N, K)
     for M, N, K in unsplit:
         assert wq.linear_workspace_size(M, N, K, wq.WQ_FMT_INT4) == 0, (M, N, K)
-    # 512 x 256 x 11008: 8 tiles of 128 x 128, 7 CTAs per tile (172 k-blocks / 24), fp32
-    # partial tiles plus one counter per tile (each part 256-byte aligned)
-    tiles, splits = 8, 7
+    # 512 x 256 x 11008: 8 tiles of 128 x 128, 8 CTAs per tile (the cap; 172 k-blocks / 8
+    # would allow 21), fp32 partial tiles plus one counter per tile (each part 256-byte aligned)
+    tiles, splits = 8, 8
     part = tiles * splits * 128 * 128 * 4
     assert wq.linear_workspace_size(512, 256, 11008, wq.WQ_FMT_INT4) == part + 256

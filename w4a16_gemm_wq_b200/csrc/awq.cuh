@@ -128,14 +128,14 @@ __global__ void __launch_bounds__(kQuantThreads) awq_delta_kernel(const uint16_t
 
 // ------------------------------------------------------------------ diagonal proxy, all alphas at once
 // Without calibration tokens the loss of alpha_i is sum_{n,k} (a_k Delta_i[n,k])^2
-// and needs W only: one pass over W evaluates every alpha.  A CTA keeps 8 rows x
+// and needs W only: one pass over W evaluates every alpha.  A CTA keeps 4 rows x
 // 1024 k of W in registers and loops over the alphas (s and 1/s per alpha from a
 // small table that stays in L2), so W is read from HBM once instead of once per
 // alpha.  The codes take the quantizer's decisions: rint(w'/scale) through a
 // reciprocal, with the IEEE division where the product lies near a rounding tie.
 // Delta = w - deq * (1/s) in fp32 and the squares are summed per thread in fp32,
 // then in fp64 across the CTA in a fixed order, one partial per (alpha, CTA).
-constexpr int kAwqProxyRows = 8;
+constexpr int kAwqProxyRows = 4;
 constexpr int kAwqProxyThreads = 128;   // 128 x 8 = 1024 k per CTA
 constexpr int kAwqProxyMaxAlphas = 32;
 
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(256) awq_proxy_table_kernel(const double* __re
   }
 }
 
-// grid = (ceil(K / 1024), ceil(N / 8)); partials[i * P + p0 + blockIdx.y * gridDim.x + blockIdx.x].
+// grid = (ceil(K / 1024), ceil(N / 4)); partials[i * P + p0 + blockIdx.y * gridDim.x + blockIdx.x].
 template <int G>
 __global__ void __launch_bounds__(kAwqProxyThreads) awq_proxy_kernel(const uint16_t* __restrict__ W, int64_t N,
                                                                      int64_t K, const float* __restrict__ tab,

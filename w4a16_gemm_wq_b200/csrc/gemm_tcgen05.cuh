@@ -15,8 +15,8 @@
 //   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
 //               (M=128, N=BN, K=16, four per k-block), tcgen05.commit frees
 //               the stage and finally signals the epilogue;
-//   warps 4..   BN dequantizer threads, one weight row each: unpack 64
-//               codes of the stage to bf16 (INT4: (q - z) * scale; NVFP4:
+//   warps 4..   2 BN dequantizer threads, two per weight row (32 k each):
+//               unpack the stage's codes to bf16 (INT4: (q - z) * scale; NVFP4:
 //               e2m1 * e4m3 block scale, the fp32 tensor scale is applied in
 //               the epilogue) and store them in the canonical K-major
 //               128-byte-swizzled layout the MMA reads; then, after the last
@@ -48,10 +48,10 @@ struct GemmShape {
   static constexpr int B_BYTES = BN * kGemmBK * 2;       // dequantized W tile
   static constexpr int P_BYTES = BN * kGemmBK / 2;       // packed 4-bit W tile
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
-  // dequantizer (then epilogue) threads: two per weight row (each 32 of a k-block's
-  // 64 k) for 128-row W tiles, so that 8 warps hide the dequantization's dependency
-  // chains; one per row for 256-row tiles; the bf16-B mode only needs the epilogue
-  static constexpr int DEQ_SPLIT = (TMA_B || BN == 256) ? 1 : 2;
+  // dequantizer (then epilogue) threads: two per weight row, each 32 of a k-block's
+  // 64 k, so that 8 or 16 warps hide the dequantization's dependency chains; the
+  // bf16-B mode only needs the epilogue warps
+  static constexpr int DEQ_SPLIT = TMA_B ? 1 : 2;
   static constexpr int DEQ_THREADS = DEQ_SPLIT * BN;
   static constexpr int THREADS = 128 + DEQ_THREADS;
   static constexpr int BAR_BYTES = 256;

@@ -284,8 +284,8 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // Plan of a quantized GEMM: the tile (see launch_gemm) and, when its CTAs
 // would cover under half of the SMs, how many CTAs share each output tile
-// along K (each at least 24 k-blocks) with the fp32 partials and per-tile
-// counters they need.
+// along K (each at least 24 k-blocks, 8 under a quarter of the SMs) with the
+// fp32 partials and per-tile counters they need.
 struct GemmPlan {
   int bn, bmt, splitk;
   int64_t tiles;
@@ -304,9 +304,14 @@ GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K) {
   p.tiles = tiles(p.bmt, p.bn);
   const int64_t nkb = (K + wq::kGemmBK - 1) / wq::kGemmBK;
   int64_t s = 1;
-  // at least 24 k-blocks per CTA: shorter K ranges lose more to the per-CTA start
-  // and the partial traffic than they gain (measured: K = 2048 slower split)
-  if (p.tiles < wq::kTcMaxCtas / 2) s = std::max<int64_t>(1, std::min<int64_t>({wq::kTcMaxCtas / p.tiles, 8, nkb / 24}));
+  // at least 24 k-blocks per CTA when the tiles cover a quarter to a half of the SMs
+  // (shorter K ranges lose more to the per-CTA start and the partial traffic than
+  // they gain: K = 2048 measured slower split there); at least 8 when they cover
+  // under a quarter (k/v_proj at M = 2048: 32 tiles would leave 116 SMs idle)
+  if (p.tiles < wq::kTcMaxCtas / 2) {
+    const int64_t floor_kb = p.tiles < wq::kTcMaxCtas / 4 ? 8 : 24;
+    s = std::max<int64_t>(1, std::min<int64_t>({wq::kTcMaxCtas / p.tiles, 8, nkb / floor_kb}));
+  }
   p.splitk = int(s);
   p.part_bytes = s > 1 ? align256(size_t(p.tiles) * size_t(s) * size_t(p.bmt) * size_t(p.bn) * 4) : 0;
   p.ws_bytes = s > 1 ? p.part_bytes + align256(size_t(p.tiles) * 4) : 0;
@@ -355,7 +360,7 @@ struct AwqLayout {
 
 // Without tokens and with at most kAwqProxyMaxAlphas alphas the search runs the
 // all-alpha proxy kernel: partial slots for up to 64 stacked matrices (each
-// starts a new 8-row block), and the s / 1/s / a table in place of Delta.
+// starts a new 4-row block), and the s / 1/s / a table in place of Delta.
 bool awq_fused_proxy(bool has_x, int n_alpha) { return !has_x && n_alpha <= wq::kAwqProxyMaxAlphas; }
 int64_t awq_proxy_kx(int64_t K) { return (K / 8 + wq::kAwqProxyThreads - 1) / wq::kAwqProxyThreads; }
 
@@ -723,6 +728,26 @@ FacLayout fac_layout(int64_t K, int64_t T) {
   return L;
 }
 
+constexpr int kMaxDevicesFac = 64;
+// A second stream per device for the factor's inverse, created on first use
+// (the library's only other per-device state besides the error word and the
+// no-allocation scratch).
+std::mutex g_fac_mu;
+cudaStream_t g_fac_stream[kMaxDevicesFac] = {};
+
+int fac_aux_stream(cudaStream_t* out) {
+  int dev = 0;
+  if (int e = cuda_check(cudaGetDevice(&dev), "cudaGetDevice")) return e;
+  if (dev < 0 || dev >= kMaxDevicesFac) return fail(WQ_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_fac_mu);
+  if (!g_fac_stream[dev]) {
+    if (int e = cuda_check(cudaStreamCreateWithFlags(&g_fac_stream[dev], cudaStreamNonBlocking), "stream create"))
+      return e;
+  }
+  *out = g_fac_stream[dev];
+  return WQ_OK;
+}
+
 int fac_gemm(const wq::FacGemmArgs& a, bool lower, cudaStream_t st) {
   static std::atomic<uint64_t> done_all{0}, done_lower{0};
   const int64_t tiles = lower ? int64_t(a.mt) * (a.mt + 1) / 2 : int64_t(a.mt) * a.nt;
@@ -960,56 +985,81 @@ int wq_gptq_hessian_factor(const uint16_t* X, int64_t T, int64_t K, double damp,
   if (int e = fac_gemm(fac_args(Xr, Tp, Xr, Tp, A, Kp, Kp, Kp, Tp, 2.0, 0.0), true, st)) return e;
   wq::fac_damp_kernel<<<1, 256, 0, st>>>(A, K, Kp, damp);
   if (int e = launched("factor damping launch")) return e;
-  // 2. blocked Cholesky of H' in place: 64-wide steps inside 256-wide super-panels;
-  // within a super-panel each step updates only the super-panel's later columns,
-  // and the rest of the trailing matrix takes one update per super-panel with a
-  // reduction depth of 256 (a quarter of the trailing-matrix traffic of
-  // updating it at every 64-wide step)
+  // 2 and 3 run on two streams: the inverse of a 256-wide super-panel (Z's columns of
+  // it) needs only that super-panel's factor (its diagonal-block inverses and its L
+  // panel, final once its 64-wide steps are done), so it overlaps the rest of the
+  // factorisation.  The inverse's stream joins the caller's before U is written,
+  // also when a launch fails, so no work outlives the call's use of the workspace.
+  cudaStream_t zs = nullptr;
+  if (int e = fac_aux_stream(&zs)) return e;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if (int e = cuda_check(cudaEventCreateWithFlags(&fork, cudaEventDisableTiming), "event create")) return e;
+  if (int e = cuda_check(cudaEventCreateWithFlags(&join, cudaEventDisableTiming), "event create")) {
+    cudaEventDestroy(fork);
+    return e;
+  }
+  const auto to_z = [&]() -> int {  // the inverse's stream waits for the work enqueued so far
+    if (int e = cuda_check(cudaEventRecord(fork, st), "event record")) return e;
+    return cuda_check(cudaStreamWaitEvent(zs, fork, 0), "stream wait");
+  };
   const int64_t SB = 4 * B;
-  for (int64_t KB = 0; KB < Kp; KB += SB) {
-    const int64_t E = std::min(KB + SB, Kp);
-    for (int64_t kb = KB; kb < E; kb += B) {
-      const int64_t e = kb + B, rest = Kp - e;
-      double* Di = Dinv + (kb / B) * B * B;
-      wq::fac_diag_kernel<<<1, 256, 0, st>>>(A, Kp, kb, Di);
-      if (int er = launched("factor diagonal block launch")) return er;
-      if (rest == 0) break;
-      double* P = A + e * Kp + kb;  // panel [rest, B]
-      if (int er = fac_gemm(fac_args(P, Kp, Di, B, P, Kp, rest, B, B, 1.0, 0.0), false, st)) return er;
-      if (e < E) {
-        if (int er = fac_gemm(fac_args(P, Kp, P, Kp, A + e * Kp + e, Kp, rest, E - e, B, -1.0, 1.0), false, st))
+  const auto factor_and_invert = [&]() -> int {
+    // Z's bytes also hold Xr, read by the Hessian product: Z is initialised after it
+    if (int e = to_z()) return e;
+    wq::fac_eye_kernel<<<unsigned(std::min<int64_t>((Kp * Kp + 255) / 256, 148 * 16)), 256, 0, zs>>>(Z, Kp);
+    if (int e = launched("factor identity launch")) return e;
+    for (int64_t KB = 0; KB < Kp; KB += SB) {
+      const int64_t E = std::min(KB + SB, Kp);
+      // 2. Cholesky of the super-panel: 64-wide steps, each updating only the
+      // super-panel's later columns
+      for (int64_t kb = KB; kb < E; kb += B) {
+        const int64_t e = kb + B, rest = Kp - e;
+        double* Di = Dinv + (kb / B) * B * B;
+        wq::fac_diag_kernel<<<1, 256, 0, st>>>(A, Kp, kb, Di);
+        if (int er = launched("factor diagonal block launch")) return er;
+        if (rest == 0) break;
+        double* P = A + e * Kp + kb;  // panel [rest, B]
+        if (int er = fac_gemm(fac_args(P, Kp, Di, B, P, Kp, rest, B, B, 1.0, 0.0), false, st)) return er;
+        if (e < E) {
+          if (int er = fac_gemm(fac_args(P, Kp, P, Kp, A + e * Kp + e, Kp, rest, E - e, B, -1.0, 1.0), false, st))
+            return er;
+        }
+      }
+      // 3. this super-panel's part of Z = L'^-T, on the inverse's stream
+      if (int e = to_z()) return e;
+      for (int64_t kb = KB; kb < E; kb += B) {
+        const int64_t e = kb + B;
+        const double* Di = Dinv + (kb / B) * B * B;
+        if (int er = fac_gemm(fac_args(Z + kb, Kp, Di, B, Z + kb, Kp, e, B, B, 1.0, 0.0), false, zs)) return er;
+        if (e < E) {
+          if (int er = fac_gemm(fac_args(Z + kb, Kp, A + e * Kp + kb, Kp, Z + e, Kp, e, E - e, B, -1.0, 1.0), false,
+                                zs))
+            return er;
+        }
+      }
+      if (E < Kp) {
+        // rows [e, E) of the super-panel's columns of Z are still 0 (Z is upper
+        // triangular), so the update may span rows 0..E with the reduction over all its columns
+        if (int er = fac_gemm(fac_args(Z + KB, Kp, A + E * Kp + KB, Kp, Z + E, Kp, E, Kp - E, E - KB, -1.0, 1.0),
+                              false, zs))
+          return er;
+        // the rest of the trailing matrix: one update with a reduction depth of 256
+        // (a quarter of the trailing-matrix traffic of an update per 64-wide step)
+        const double* Q = A + E * Kp + KB;  // [Kp - E, E - KB]
+        if (int er = fac_gemm(fac_args(Q, Kp, Q, Kp, A + E * Kp + E, Kp, Kp - E, Kp - E, E - KB, -1.0, 1.0), true, st))
           return er;
       }
     }
-    if (E < Kp) {
-      const double* Q = A + E * Kp + KB;  // [Kp - E, E - KB]
-      if (int er = fac_gemm(fac_args(Q, Kp, Q, Kp, A + E * Kp + E, Kp, Kp - E, Kp - E, E - KB, -1.0, 1.0), true, st))
-        return er;
-    }
-  }
-  // 3. Z = L'^-T by blocked substitution, with the same two-level blocking
-  wq::fac_eye_kernel<<<unsigned(std::min<int64_t>((Kp * Kp + 255) / 256, 148 * 16)), 256, 0, st>>>(Z, Kp);
-  if (int e = launched("factor identity launch")) return e;
-  for (int64_t KB = 0; KB < Kp; KB += SB) {
-    const int64_t E = std::min(KB + SB, Kp);
-    for (int64_t kb = KB; kb < E; kb += B) {
-      const int64_t e = kb + B;
-      const double* Di = Dinv + (kb / B) * B * B;
-      if (int er = fac_gemm(fac_args(Z + kb, Kp, Di, B, Z + kb, Kp, e, B, B, 1.0, 0.0), false, st)) return er;
-      if (e < E) {
-        if (int er = fac_gemm(fac_args(Z + kb, Kp, A + e * Kp + kb, Kp, Z + e, Kp, e, E - e, B, -1.0, 1.0), false,
-                              st))
-          return er;
-      }
-    }
-    if (E < Kp) {
-      // rows [e, E) of the super-panel's columns are still 0 (Z is upper triangular), so
-      // the update may span rows 0..E with the reduction over all its columns
-      if (int er = fac_gemm(fac_args(Z + KB, Kp, A + E * Kp + KB, Kp, Z + E, Kp, E, Kp - E, E - KB, -1.0, 1.0),
-                            false, st))
-        return er;
-    }
-  }
+    return WQ_OK;
+  };
+  const int err = factor_and_invert();
+  // join (always): the caller's stream waits for everything enqueued on the inverse's stream
+  int jerr = cuda_check(cudaEventRecord(join, zs), "event record");
+  if (!jerr) jerr = cuda_check(cudaStreamWaitEvent(st, join, 0), "stream wait");
+  cudaEventDestroy(fork);
+  cudaEventDestroy(join);
+  if (err) return err;
+  if (jerr) return jerr;
   // 4. U from Z, reversed and transposed, fp32
   const unsigned kt = unsigned((K + 31) / 32);
   wq::fac_u_kernel<<<dim3(kt, kt), 256, 0, st>>>(Z, K, Kp, U);
