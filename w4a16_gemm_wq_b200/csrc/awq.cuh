@@ -217,16 +217,31 @@ __global__ void __launch_bounds__(kAwqProxyThreads) awq_proxy_kernel(const uint1
       if (!rin[r]) continue;  // whole groups share rin (a group never straddles rows or K)
       float sc;
       group_scale_f16(__fsub_rn(mx, mn), 15.0f, &sc);
-      const float z = fminf(fmaxf(rintf(__fdiv_rn(-mn, sc)), 0.0f), 15.0f);
       const float rsc = __frcp_rn(sc);
+      // z = rint(-mn / sc) and q = rint(wp / sc) through the reciprocal: |t - x / sc|
+      // <= ~2^-22 |t| with |t| <= ~16, so rint(t) is the quotient's rint unless t lies
+      // within 1e-5 of a half-integer; those few take the division in a branch of
+      // their own (not issued, predicated off, for every weight)
+      const float tz = __fmul_rn(-mn, rsc);
+      float zr = rintf(tz);
+      float qr[8];
+      uint32_t slow = fabsf(0.5f - fabsf(__fsub_rn(tz, zr))) < 1e-5f ? 0x100u : 0u;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        // |t - wp / sc| <= ~2^-22 |t| with |t| <= ~16: rint(t) is the quotient's rint
-        // unless t lies within 1e-5 of a half-integer
         const float t = __fmul_rn(wp[j], rsc);
-        float q = rintf(t);
-        if (fabsf(fabsf(t - truncf(t)) - 0.5f) < 1e-5f) q = rintf(__fdiv_rn(wp[j], sc));
-        q = fminf(fmaxf(__fadd_rn(q, z), 0.0f), 15.0f);
+        qr[j] = rintf(t);
+        if (fabsf(0.5f - fabsf(__fsub_rn(t, qr[j]))) < 1e-5f) slow |= 1u << j;
+      }
+      if (__builtin_expect(slow != 0, 0)) {
+        if (slow & 0x100u) zr = rintf(__fdiv_rn(-mn, sc));
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (slow & (1u << j)) qr[j] = rintf(__fdiv_rn(wp[j], sc));
+      }
+      const float z = fminf(fmaxf(zr, 0.0f), 15.0f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float q = fminf(fmaxf(__fadd_rn(qr[j], z), 0.0f), 15.0f);
         const float deq = __fmul_rn(__fsub_rn(q, z), sc);
         const float v = __fmul_rn(av[j], __fsub_rn(w[j], __fmul_rn(deq, rv[j])));
         sq = __fmaf_rn(v, v, sq);

@@ -98,15 +98,27 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_int4_kernel(
     uint32_t word = 0;
     // rint(w / sc) through the correctly rounded reciprocal: t = w * (1 / sc) is
     // within 2^-23 |t| of the IEEE quotient, so its rint is the quotient's unless t
-    // lies within 2^-21 |t| of a half-integer, where the division itself is taken
+    // lies within 2^-21 |t| of a half-integer, where the division itself is taken.
+    // Those (rare) weights are flagged and divided in a branch of their own, so
+    // the division sequence is not issued, predicated off, for every weight.
     const float rsc = __frcp_rn(sc);
+    float r[8];
+    uint32_t slow = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float t = __fmul_rn(w[j], rsc);
-      float r = rintf(t);
-      if (fabsf(fabsf(__fsub_rn(t, truncf(t))) - 0.5f) <= fabsf(t) * 0x1p-21f) r = rintf(__fdiv_rn(w[j], sc));
-      const float q = ASYM ? fminf(fmaxf(__fadd_rn(r, z), 0.0f), 15.0f)
-                           : __fadd_rn(fminf(fmaxf(r, -7.0f), 7.0f), 8.0f);
+      r[j] = rintf(t);
+      if (fabsf(0.5f - fabsf(__fsub_rn(t, r[j]))) <= fabsf(t) * 0x1p-21f) slow |= 1u << j;
+    }
+    if (__builtin_expect(slow != 0, 0)) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (slow & (1u << j)) r[j] = rintf(__fdiv_rn(w[j], sc));
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float q = ASYM ? fminf(fmaxf(__fadd_rn(r[j], z), 0.0f), 15.0f)
+                           : __fadd_rn(fminf(fmaxf(r[j], -7.0f), 7.0f), 8.0f);
       word |= uint32_t(q) << (4 * j);
     }
     qweight[n * words + u] = word;
@@ -243,16 +255,24 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(const uint16_t* __restr
       // pairs near a rounding boundary take the divisions.  A denominator below
       // 2^-128 (tensors with amax under ~1e-33) has no finite reciprocal: then
       // every pair takes the divisions.
+      // Pairs that take the divisions are flagged and converted in a branch of
+      // their own (rare), so the divisions are not issued, predicated off, for all.
       const bool rcp_ok = __float_as_uint(rcp) < 0x7F800000u;
       uint32_t pairs[8];
+      uint32_t slow = 0;
 #pragma unroll
       for (int j = 0; j < 16; j += 2) {
         const float t0 = __fmul_rn(w[j], rcp), t1 = __fmul_rn(w[j + 1], rcp);
         const uint32_t c = e2m1x2_rn_sat(t0, t1);
         const uint32_t cl = e2m1x2_rn_sat(__fmul_rn(t0, 1.0f - 0x1p-19f), __fmul_rn(t1, 1.0f - 0x1p-19f));
         const uint32_t ch = e2m1x2_rn_sat(__fmul_rn(t0, 1.0f + 0x1p-19f), __fmul_rn(t1, 1.0f + 0x1p-19f));
-        pairs[j >> 1] = (rcp_ok && c == cl && c == ch) ? c
-                                                         : e2m1x2_rn_sat(__fdiv_rn(w[j], denom), __fdiv_rn(w[j + 1], denom));
+        pairs[j >> 1] = c;
+        if (!(rcp_ok && c == cl && c == ch)) slow |= 1u << (j >> 1);
+      }
+      if (__builtin_expect(slow != 0, 0)) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (slow & (1u << q)) pairs[q] = e2m1x2_rn_sat(__fdiv_rn(w[2 * q], denom), __fdiv_rn(w[2 * q + 1], denom));
       }
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
