@@ -225,12 +225,12 @@ __global__ void __launch_bounds__(kAwqProxyThreads) awq_proxy_kernel(const uint1
       const float tz = __fmul_rn(-mn, rsc);
       float zr = rintf(tz);
       float qr[8];
-      uint32_t slow = fabsf(0.5f - fabsf(__fsub_rn(tz, zr))) < 1e-5f ? 0x100u : 0u;
+      uint32_t slow = __fsub_rn(0.5f, fabsf(__fsub_rn(tz, zr))) < 1e-5f ? 0x100u : 0u;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const float t = __fmul_rn(wp[j], rsc);
         qr[j] = rintf(t);
-        if (fabsf(0.5f - fabsf(__fsub_rn(t, qr[j]))) < 1e-5f) slow |= 1u << j;
+        if (__fsub_rn(0.5f, fabsf(__fsub_rn(t, qr[j]))) < 1e-5f) slow |= 1u << j;  // |t - rint(t)| <= 0.5
       }
       if (__builtin_expect(slow != 0, 0)) {
         if (slow & 0x100u) zr = rintf(__fdiv_rn(-mn, sc));
@@ -238,11 +238,11 @@ __global__ void __launch_bounds__(kAwqProxyThreads) awq_proxy_kernel(const uint1
         for (int j = 0; j < 8; ++j)
           if (slow & (1u << j)) qr[j] = rintf(__fdiv_rn(wp[j], sc));
       }
-      const float z = fminf(fmaxf(zr, 0.0f), 15.0f);
+      // q - z = clamp(rint + z, 0, 15) - z = clamp(rint, -z, 15 - z), exactly (small integers)
+      const float z = fminf(fmaxf(zr, 0.0f), 15.0f), lo_q = -z, hi_q = __fsub_rn(15.0f, z);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const float q = fminf(fmaxf(__fadd_rn(qr[j], z), 0.0f), 15.0f);
-        const float deq = __fmul_rn(__fsub_rn(q, z), sc);
+        const float deq = __fmul_rn(fminf(fmaxf(qr[j], lo_q), hi_q), sc);
         const float v = __fmul_rn(av[j], __fsub_rn(w[j], __fmul_rn(deq, rv[j])));
         sq = __fmaf_rn(v, v, sq);
       }
