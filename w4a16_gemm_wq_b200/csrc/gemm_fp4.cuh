@@ -63,6 +63,8 @@ struct Fp4Args {
   const float* gx;        // fp32 [1]
   const float* gw;        // fp32 [1]
   uint16_t* Y;            // bf16 [M, N]
+  CUtensorMap tmY;        // Y bf16 [M, N], box {32, 32}, 64B swizzle (persistent kernel, used iff y_tma)
+  int y_tma;              // N % 8 == 0 and Y 16-byte aligned: the epilogue stores Y tiles by TMA
   int M, N, K;            // K % 64 == 0
 };
 
@@ -347,7 +349,9 @@ struct Fp4PShape {
   static constexpr int ACC_COLS = 2 * kFp4PBN;
   static constexpr int TMEM_COLS = 512;
   static_assert(ACC_COLS + STAGES * SF_STAGE_COLS <= TMEM_COLS, "tensor memory budget");
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+  static constexpr int YBOX_BYTES = 32 * 32 * 2;      // one epilogue warp's 32 x 32 bf16 box of Y
+  static constexpr int Y_BYTES = 4 * 2 * YBOX_BYTES;  // two boxes per epilogue warp (store / fill)
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + Y_BYTES + 256 + 1024;
   static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled tiles");
 };
 
@@ -359,7 +363,8 @@ __global__ void __launch_bounds__(Fp4PShape::THREADS, 1) gemm_fp4_persistent_ker
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+  uint8_t* ybox = smem + STAGES * S::STAGE_BYTES;  // epilogue Y boxes (1024-byte aligned)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ybox + S::Y_BYTES);
   uint64_t* full = bars;                    // TMA landed (codes + scales)
   uint64_t* sfready = bars + STAGES;        // scales in tensor memory
   uint64_t* empty = bars + 2 * STAGES;      // MMAs of the stage finished
@@ -389,6 +394,7 @@ __global__ void __launch_bounds__(Fp4PShape::THREADS, 1) gemm_fp4_persistent_ker
     prefetch_tmap(&a.tmB);
     prefetch_tmap(&a.tmSA);
     prefetch_tmap(&a.tmSB);
+    if (a.y_tma) prefetch_tmap(&a.tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -493,7 +499,7 @@ __global__ void __launch_bounds__(Fp4PShape::THREADS, 1) gemm_fp4_persistent_ker
     const uint32_t lane_base = uint32_t(quarter * 32) << 16;
     const float gmul = __ldg(a.gx) * __ldg(a.gw);
     const bool vec = (a.N % 8) == 0;
-    int i = 0;
+    int i = 0, nbox = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       const int b = i & 1, u = i >> 1;
       bool go = mbar_wait(&acc_full[b], u & 1, ERR_TIMEOUT_MMA, abort_flag);
@@ -505,6 +511,32 @@ __global__ void __launch_bounds__(Fp4PShape::THREADS, 1) gemm_fp4_persistent_ker
       for (int c = 0; c < BN; c += 32) {
         uint32_t v[32];
         tmem_ld32(tmem + lane_base + uint32_t(b * BN + c), v);
+        if (a.y_tma) {
+          // the warp's 32 x 32 box (row = lane) through shared memory and one TMA
+          // store: full 128-byte lines to L2 instead of 16-byte pieces of 32 rows.
+          // Box buffers alternate; the one used two boxes ago must have been read.
+          uint8_t* box = ybox + (quarter * 2 + (nbox & 1)) * S::YBOX_BYTES;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          const uint32_t rbase = smem_u32(box) + uint32_t(lane * 64);
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {  // 16-byte piece qq of the row, at its 64B-swizzled place
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v[8 * qq + 0]) * gmul, __uint_as_float(v[8 * qq + 1]) * gmul);
+            o.y = pack_bf16x2(__uint_as_float(v[8 * qq + 2]) * gmul, __uint_as_float(v[8 * qq + 3]) * gmul);
+            o.z = pack_bf16x2(__uint_as_float(v[8 * qq + 4]) * gmul, __uint_as_float(v[8 * qq + 5]) * gmul);
+            o.w = pack_bf16x2(__uint_as_float(v[8 * qq + 6]) * gmul, __uint_as_float(v[8 * qq + 7]) * gmul);
+            st_shared_v4(rbase + uint32_t((qq ^ ((lane >> 1) & 3)) << 4), o);
+          }
+          fence_proxy_async_smem();  // generic-proxy stores -> visible to the TMA
+          __syncwarp();
+          if (lane == 0) {  // rows or columns past M / N are clipped by the TMA
+            tma_store_2d(&a.tmY, box, n0 + c, m0 + quarter * 32);
+            bulk_commit();
+          }
+          ++nbox;
+          continue;
+        }
         if (row < a.M) {
           uint16_t* yrow = a.Y + int64_t(row) * a.N;
           const int nb = n0 + c;
@@ -528,6 +560,7 @@ __global__ void __launch_bounds__(Fp4PShape::THREADS, 1) gemm_fp4_persistent_ker
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
+    if (lane == 0) bulk_wait_all();  // the Y stores are complete before the CTA leaves
   }
   tc_fence_before();
   __syncthreads();

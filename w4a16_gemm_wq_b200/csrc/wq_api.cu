@@ -413,6 +413,13 @@ int launch_fp4_persistent(wq::Fp4Args& a, const uint8_t* wcodes, cudaStream_t st
   if (int e = make_tmap_2d(&a.tmSB, a.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 16),
                            wq::kFp4PBN, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
     return e;
+  // the epilogue stores Y by TMA when its rows are 16-byte aligned
+  a.y_tma = (a.N % 8 == 0) && aligned16(a.Y);
+  if (a.y_tma) {
+    if (int e = make_tmap_2d(&a.tmY, a.Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(a.M), uint64_t(a.N), 32, 32,
+                             CU_TENSOR_MAP_SWIZZLE_64B))
+      return e;
+  }
   static std::atomic<uint64_t> attr_done{0};
   if (int e = ensure_smem_attr(wq::gemm_fp4_persistent_kernel, S::SMEM_BYTES, &attr_done,
                                "fp4 persistent smem attribute"))
