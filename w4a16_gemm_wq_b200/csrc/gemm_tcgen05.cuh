@@ -71,6 +71,8 @@ struct GemmArgs {
   const float* gscale;      // NVFP4 fp32 [1]
   const float* inv_s;       // fp32 [K] or null
   uint16_t* Y;              // bf16 [M, N]
+  CUtensorMap tmY;          // Y bf16 [M, N], box {32, 32}, 64B swizzle (used iff y_tma)
+  int y_tma;                // unsplit INT4 / NVFP4 with N % 8 == 0 and Y 16-byte aligned: Y boxes by TMA
   double* sq_partials;      // FMT_BF16_SQ: one partial sum of squares per epilogue warp
   float* part;              // split-K: fp32 partial tiles [tiles][splitk][BMT * BN]
   unsigned* ctr;            // split-K: arrivals per tile (0 before and after a launch)
@@ -275,6 +277,7 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT, FMT == GEMM_BF16_SQ>::THREA
     fence_mbar_init();
     prefetch_tmap(&a.tmA);
     prefetch_tmap(&a.tmP);
+    if (a.y_tma) prefetch_tmap(&a.tmY);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -528,12 +531,40 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT, FMT == GEMM_BF16_SQ>::THREA
       tc_fence_after();
       const float gmul = (FMT == GEMM_NVFP4) ? __ldg(a.gscale) : 1.0f;
       double sq = 0.0;
+      int nbox = 0;
       // (accumulator, 32-column chunk) units of this quarter, dealt round-robin
       for (int u = wi; u < S::NACC * (BN / 32); u += WPQ) {
         const int acc = u / (BN / 32), c = (u % (BN / 32)) * 32;
         const int row = m0 + acc * kGemmBM + quarter * 32 + lane;
         uint32_t v[32];
         tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN + c), v);
+        if (FMT != GEMM_BF16_SQ && a.y_tma) {
+          // the unit's 32 x 32 box (row = lane) through shared memory and one TMA store
+          // (full lines to L2).  Every k-block's MMAs completed, so the stage buffers
+          // are free: each epilogue warp takes two 2 KB boxes of them, alternating; the
+          // one used two boxes ago must have been read.
+          uint8_t* box = smem + ((warp - DEQ_WARP0) * 2 + (nbox & 1)) * 2048;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          const uint32_t rbase = smem_u32(box) + uint32_t(lane * 64);
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {  // 16-byte piece qq of the row, at its 64B-swizzled place
+            uint4 o;
+            o.x = pack_bf16x2(__uint_as_float(v[8 * qq + 0]) * gmul, __uint_as_float(v[8 * qq + 1]) * gmul);
+            o.y = pack_bf16x2(__uint_as_float(v[8 * qq + 2]) * gmul, __uint_as_float(v[8 * qq + 3]) * gmul);
+            o.z = pack_bf16x2(__uint_as_float(v[8 * qq + 4]) * gmul, __uint_as_float(v[8 * qq + 5]) * gmul);
+            o.w = pack_bf16x2(__uint_as_float(v[8 * qq + 6]) * gmul, __uint_as_float(v[8 * qq + 7]) * gmul);
+            st_shared_v4(rbase + uint32_t((qq ^ ((lane >> 1) & 3)) << 4), o);
+          }
+          fence_proxy_async_smem();  // generic-proxy stores -> visible to the TMA
+          __syncwarp();
+          if (lane == 0) {  // rows or columns past M / N are clipped by the TMA
+            tma_store_2d(&a.tmY, box, n0 + c, m0 + acc * kGemmBM + quarter * 32);
+            bulk_commit();
+          }
+          ++nbox;
+          continue;
+        }
         if (FMT == GEMM_BF16_SQ) {
           float part = 0.f;
           if (row < a.M) {
@@ -576,6 +607,7 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT, FMT == GEMM_BF16_SQ>::THREA
       }
     }
   }
+  if (FMT != GEMM_BF16_SQ && a.y_tma && warp >= DEQ_WARP0 && lane == 0) bulk_wait_all();  // Y boxes stored
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -270,6 +270,13 @@ int launch_gemm_bn(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaS
   if (int e = make_tmap_2d(&a.tmP, packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, uint64_t(a.N), uint64_t(a.K / 2), BN,
                            wq::kGemmBK / 2, CU_TENSOR_MAP_SWIZZLE_NONE))
     return e;
+  // unsplit products store Y by TMA when its rows are 16-byte aligned
+  a.y_tma = a.splitk <= 1 && (a.N % 8 == 0) && aligned16(a.Y);
+  if (a.y_tma) {
+    if (int e = make_tmap_2d(&a.tmY, a.Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(a.M), uint64_t(a.N), 32, 32,
+                             CU_TENSOR_MAP_SWIZZLE_64B))
+      return e;
+  }
   return launch_gemm_prepared<FMT, BN, BMT>(a, st);
 }
 
