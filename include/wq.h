@@ -92,8 +92,9 @@ int wq_nvfp4_sizes(int64_t N, int64_t K, size_t* codes_bytes, size_t* bscale_byt
  * workspace of this size.  W4A16 never requires one: a non-zero size means a
  * prefill GEMM with few output tiles (under half the SMs) that, given a
  * workspace of at least this size, splits K over several CTAs per tile (fp32
- * partials summed in split order by the last CTA of each tile, so the result
- * does not depend on timing); with ws = NULL or a smaller one it runs unsplit. */
+ * partial tiles, then a reduction launch that sums them in split order, so the
+ * result does not depend on timing); with ws = NULL or a smaller one it runs
+ * unsplit. */
 int wq_linear_workspace_size(int64_t M, int64_t N, int64_t K, int format, int act_fp4,
                              size_t* bytes);
 

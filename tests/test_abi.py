@@ -107,18 +107,20 @@ def test_gptq_and_shared_awq_validate_on_the_host(lib):
 
 
 def test_split_k_plan_is_host_logic():
-    # the prefill GEMM splits K only when its tiles cover under half of the SMs: at
-    # least 24 k-blocks per split for 37..73 tiles, at least 8 for fewer; the workspace
-    # query is the plan's size and 0 when nothing splits
-    split = [(512, 256, 11008), (512, 2048, 11008), (2048, 256, 4096), (512, 256, 2048)]
-    unsplit = [(512, 2048, 2048), (8192, 11008, 2048), (2048, 2048, 2048), (16, 256, 11008)]
+    # the prefill GEMM's plan (tile and split count from a cost model of CTA rates) is
+    # host logic: K splits only where the tiles leave SMs idle and K is long enough; the
+    # workspace query is the partial tiles' size (whole fp32 tiles, one wave of CTAs at
+    # most) and 0 when nothing splits
+    split = [(512, 256, 11008), (512, 2048, 11008), (2048, 256, 4096), (512, 256, 2048), (512, 2048, 2048),
+             (2048, 2048, 11008)]
+    unsplit = [(8192, 11008, 2048), (2048, 2048, 2048), (16, 256, 11008), (512, 11008, 2048)]
     for M, N, K in split:
-        assert wq.linear_workspace_size(M, N, K, wq.WQ_FMT_INT4) > 0, (M, N, K)
-        assert wq.linear_workspace_size(M, N, K, wq.WQ_FMT_NVFP4) > 0, (M, N, K)
+        for fmt in (wq.WQ_FMT_INT4, wq.WQ_FMT_NVFP4):
+            ws = wq.linear_workspace_size(M, N, K, fmt)
+            assert ws > 0, (M, N, K)
+            assert ws % (128 * 128 * 4) == 0 and ws <= 148 * 256 * 256 * 4, (M, N, K, ws)
     for M, N, K in unsplit:
         assert wq.linear_workspace_size(M, N, K, wq.WQ_FMT_INT4) == 0, (M, N, K)
-    # 512 x 256 x 11008: 8 tiles of 128 x 128, 8 CTAs per tile (the cap; 172 k-blocks / 8
-    # would allow 21), fp32 partial tiles plus one counter per tile (each part 256-byte aligned)
-    tiles, splits = 8, 8
-    part = tiles * splits * 128 * 128 * 4
-    assert wq.linear_workspace_size(512, 256, 11008, wq.WQ_FMT_INT4) == part + 256
+    # the plan depends on the shape only: the same query twice, and INT4 / NVFP4 alike
+    assert wq.linear_workspace_size(512, 2048, 11008, wq.WQ_FMT_INT4) == \
+        wq.linear_workspace_size(512, 2048, 11008, wq.WQ_FMT_NVFP4)

@@ -72,10 +72,10 @@ struct GemmArgs {
   const float* inv_s;       // fp32 [K] or null
   uint16_t* Y;              // bf16 [M, N]
   CUtensorMap tmY;          // Y bf16 [M, N], box {32, 32}, 64B swizzle (used iff y_tma)
+  CUtensorMap tmPart;       // split-K partials fp32 [tiles * splitk * BMT, BN], box {32, 32}, 128B swizzle
   int y_tma;                // unsplit INT4 / NVFP4 with N % 8 == 0 and Y 16-byte aligned: Y boxes by TMA
   double* sq_partials;      // FMT_BF16_SQ: one partial sum of squares per epilogue warp
-  float* part;              // split-K: fp32 partial tiles [tiles][splitk][BMT * BN]
-  unsigned* ctr;            // split-K: arrivals per tile (0 before and after a launch)
+  float* part;              // split-K: fp32 partial tiles [tiles][splitk][BMT * BN] (split_reduce_kernel sums them)
   int splitk;               // CTAs per output tile along K (gridDim.z); 1 = no split
   int M, N, K;              // K: reduction length (for FMT_BF16_SQ the length of B's rows)
   int a_kblocks;            // A k-block index wraps modulo this (FMT_BF16_SQ reuses X twice)
@@ -254,7 +254,6 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT, FMT == GEMM_BF16_SQ>::THREA
   uint64_t* accum = bars + 3 * STAGES;   // accumulator complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* split_last = reinterpret_cast<volatile int*>(tmem_slot + 2);  // split-K: this CTA sums the tile
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * BMT, n0 = blockIdx.x * BN;
@@ -457,75 +456,36 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT, FMT == GEMM_BF16_SQ>::THREA
     const int wi = (warp - DEQ_WARP0) >> 2;            // this warp's index among them
     const bool vec = (a.N % 8) == 0;
     if (FMT != GEMM_BF16_SQ && a.splitk > 1) {
-      // split-K: store this CTA's fp32 partial tile; the CTA that arrives last at
-      // the tile's counter adds the splitk partials in split order and writes Y
-      // (no CTA waits for another; the sum's order does not depend on timing).
-      // Every epilogue warp passes both barriers, whether or not its wait succeeded.
-      const float gmul = (FMT == GEMM_NVFP4) ? __ldg(a.gscale) : 1.0f;
-      const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-      constexpr int TILE = BMT * BN;
+      // split-K: this CTA's fp32 partial tile leaves by TMA (32 x 32 boxes staged in
+      // the freed stage buffers, 128-byte swizzle); split_reduce_kernel, launched
+      // next, adds the partials in split order and writes Y (no CTA waits for
+      // another; the sum's order does not depend on timing).
       if (go) {
         tc_fence_after();
-        float* mine = a.part + (int64_t(tile) * a.splitk + blockIdx.z) * TILE;
+        const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+        const int prow0 = (tile * a.splitk + int(blockIdx.z)) * BMT;  // this partial tile's first row
+        int nbox = 0;
         for (int u = wi; u < S::NACC * (BN / 32); u += WPQ) {
           const int acc = u / (BN / 32), c = (u % (BN / 32)) * 32;
-          const int rt = acc * kGemmBM + quarter * 32 + lane;  // row within the tile
           uint32_t v[32];
           tmem_ld32(tmem_acc + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN + c), v);
-          float4* dst = reinterpret_cast<float4*>(mine + rt * BN + c);
+          uint8_t* box = smem + (warp - DEQ_WARP0) * 8192 + (nbox & 1) * 4096;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          const uint32_t rbase = smem_u32(box) + uint32_t(lane * 128);
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                 __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-        }
-      }
-      {
-        __threadfence();
-        asm volatile("bar.sync 1, %0;" ::"r"(DEQ_WARPS * 32) : "memory");  // the epilogue warps only
-        if (threadIdx.x == DEQ_WARP0 * 32)
-          *split_last = (atomicAdd(a.ctr + tile, 1u) == unsigned(a.splitk - 1)) ? 1 : 0;
-        asm volatile("bar.sync 1, %0;" ::"r"(DEQ_WARPS * 32) : "memory");
-        if (*split_last) {
-          __threadfence();
-          const float* base = a.part + int64_t(tile) * a.splitk * TILE;
-          for (int u = wi; u < S::NACC * (BN / 32); u += WPQ) {
-            const int acc = u / (BN / 32), c = (u % (BN / 32)) * 32;
-            const int rt = acc * kGemmBM + quarter * 32 + lane;
-            const int row = m0 + rt;
-            float v[32];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 x = __ldcg(reinterpret_cast<const float4*>(base + rt * BN + c) + q);
-              v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
-            }
-            for (int sp = 1; sp < a.splitk; ++sp) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 x = __ldcg(reinterpret_cast<const float4*>(base + int64_t(sp) * TILE + rt * BN + c) + q);
-                v[4 * q] += x.x; v[4 * q + 1] += x.y; v[4 * q + 2] += x.z; v[4 * q + 3] += x.w;
-              }
-            }
-            if (row < a.M) {
-              uint16_t* yrow = a.Y + int64_t(row) * a.N;
-              const int nb = n0 + c;
-              if (vec && nb + 32 <= a.N) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  uint4 o;
-                  o.x = pack_bf16x2(v[8 * q + 0] * gmul, v[8 * q + 1] * gmul);
-                  o.y = pack_bf16x2(v[8 * q + 2] * gmul, v[8 * q + 3] * gmul);
-                  o.z = pack_bf16x2(v[8 * q + 4] * gmul, v[8 * q + 5] * gmul);
-                  o.w = pack_bf16x2(v[8 * q + 6] * gmul, v[8 * q + 7] * gmul);
-                  *reinterpret_cast<uint4*>(yrow + nb + 8 * q) = o;
-                }
-              } else {
-                for (int q = 0; q < 32; ++q)
-                  if (nb + q < a.N) yrow[nb + q] = uint16_t(f32_to_bf16_bits(v[q] * gmul));
-              }
-            }
+          for (int q = 0; q < 8; ++q)  // 16-byte piece q of the row, at its 128B-swizzled place
+            st_shared_v4(rbase + uint32_t((q ^ (lane & 7)) << 4),
+                         make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&a.tmPart, box, c, prow0 + acc * kGemmBM + quarter * 32);
+            bulk_commit();
           }
-          if (threadIdx.x == DEQ_WARP0 * 32) a.ctr[tile] = 0u;  // clean for the next launch
+          ++nbox;
         }
+        if (lane == 0) bulk_wait_all();  // the partial is stored before the CTA leaves
       }
     } else if (go) {
       tc_fence_after();
@@ -614,6 +574,47 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT, FMT == GEMM_BF16_SQ>::THREA
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_acc, S::TMEM_COLS);
+  }
+}
+
+// Split-K reduction: Y[m, n] = gmul * sum over the splits, in split order, of the
+// fp32 partial tiles part[tile][split][BMT][BN] (tile = (m / BMT) * n_tiles + n / BN).
+// Each thread takes 4 consecutive columns of one tile row: every split's float4
+// load in flight at once, coalesced across the warp.  A stream-ordered successor
+// of the GEMM: it reads the partials only after griddepcontrol.wait.
+__global__ void __launch_bounds__(256) split_reduce_kernel(const float* __restrict__ part, int splitk, int bmt,
+                                                           int bn, int n_tiles, int64_t quads, int M, int N,
+                                                           const float* __restrict__ gscale, uint16_t* __restrict__ Y) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float gmul = gscale ? __ldg(gscale) : 1.0f;
+  const int64_t tile_quads = int64_t(bmt) * bn / 4;
+  for (int64_t g = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; g < quads; g += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t tile = g / tile_quads;
+    const int e = int(g - tile * tile_quads) * 4;  // element within the tile
+    const int rt = e / bn, ct = e - rt * bn;
+    const int row = int(tile / n_tiles) * bmt + rt, col = int(tile % n_tiles) * bn + ct;
+    if (row >= M || col >= N) continue;
+    const float4* src = reinterpret_cast<const float4*>(part + tile * splitk * int64_t(bmt) * bn + e);
+    const int64_t stride4 = int64_t(bmt) * bn / 4;
+    float4 x[8];
+#pragma unroll
+    for (int sp = 0; sp < 8; ++sp)
+      if (sp < splitk) x[sp] = __ldcs(src + sp * stride4);
+    float4 t = x[0];
+#pragma unroll
+    for (int sp = 1; sp < 8; ++sp)
+      if (sp < splitk) {
+        t.x += x[sp].x; t.y += x[sp].y; t.z += x[sp].z; t.w += x[sp].w;
+      }
+    uint16_t* yp = Y + int64_t(row) * N + col;
+    if ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(Y) & 7) == 0) {
+      *reinterpret_cast<uint2*>(yp) = make_uint2(pack_bf16x2(t.x * gmul, t.y * gmul), pack_bf16x2(t.z * gmul, t.w * gmul));
+    } else {
+      const float tv[4] = {t.x, t.y, t.z, t.w};
+      for (int q = 0; q < 4; ++q)
+        if (col + q < N) yp[q] = uint16_t(f32_to_bf16_bits(tv[q] * gmul));
+    }
   }
 }
 

@@ -282,74 +282,95 @@ int launch_gemm_bn(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaS
 
 int gemm_bn(int64_t M, int64_t N);
 
-// Tile of the quantized GEMM.  A 256-row CTA (two accumulators sharing each
-// dequantized W tile) does twice the flops of a 128-row one for the same
-// dequantization, so one wave of them is never slower than two waves of
-// 128-row tiles: use it while it still covers about two thirds of the SMs,
-// with the widest W tile that does; else 128 rows.
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// Plan of a quantized GEMM: the tile (see launch_gemm) and, when its CTAs
-// would cover under half of the SMs, how many CTAs share each output tile
-// along K (each at least 24 k-blocks, 8 under a quarter of the SMs) with the
-// fp32 partials and per-tile counters they need.
+// Plan of a quantized GEMM: the tile (BMT x BN) and how many CTAs share each
+// output tile along K (fp32 partial tiles, then the reduction launch), chosen by
+// a cost model fitted to measured CTA rates on B200: a CTA spends t_kb per
+// 64-deep k-block (set by its dequantization and MMA work: 0.60 us for 128 x 128,
+// 0.80 for 256 x 128, 0.85 for 128 x 256 and 256 x 256 with every SM busy)
+// plus ~3 us to start and drain; CTAs beyond one wave of 148 queue; a split adds
+// the partial tiles' HBM round trip (~5 TB/s) and a ~2 us launch.  Splits stay
+// within one wave and keep at least 4 k-blocks per CTA.  Without a workspace
+// (allow_split false) the best unsplit plan is taken.
 struct GemmPlan {
   int bn, bmt, splitk;
   int64_t tiles;
   size_t part_bytes, ws_bytes;
 };
-GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K) {
-  const auto tiles = [&](int bm, int bn) { return ((N + bn - 1) / bn) * ((M + bm - 1) / bm); };
-  GemmPlan p = {};
-  if (tiles(256, 256) >= 100) {
-    p.bn = 256; p.bmt = 256;
-  } else if (tiles(256, 128) >= 100) {
-    p.bn = 128; p.bmt = 256;
-  } else {
-    p.bn = gemm_bn(M, N); p.bmt = wq::kGemmBM;
-  }
-  p.tiles = tiles(p.bmt, p.bn);
+GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K, bool allow_split = true) {
+  struct Cfg {
+    int bmt, bn;
+    double t_kb;
+  };
+  static const Cfg cfgs[4] = {{256, 256, 0.85}, {256, 128, 0.80}, {128, 256, 0.85}, {128, 128, 0.60}};
   const int64_t nkb = (K + wq::kGemmBK - 1) / wq::kGemmBK;
-  int64_t s = 1;
-  // at least 24 k-blocks per CTA when the tiles cover a quarter to a half of the SMs
-  // (shorter K ranges lose more to the per-CTA start and the partial traffic than
-  // they gain: K = 2048 measured slower split there); at least 8 when they cover
-  // under a quarter (k/v_proj at M = 2048: 32 tiles would leave 116 SMs idle)
-  if (p.tiles < wq::kTcMaxCtas / 2) {
-    const int64_t floor_kb = p.tiles < wq::kTcMaxCtas / 4 ? 8 : 24;
-    s = std::max<int64_t>(1, std::min<int64_t>({wq::kTcMaxCtas / p.tiles, 8, nkb / floor_kb}));
+  const int64_t sms = wq::kTcMaxCtas;
+  GemmPlan best = {};
+  double best_t = 0.0;
+  for (const Cfg& c : cfgs) {
+    const int64_t tiles = ((N + c.bn - 1) / c.bn) * ((M + c.bmt - 1) / c.bmt);
+    for (int64_t sp = 1; sp <= 8; sp *= 2) {
+      if (sp > 1 && (!allow_split || tiles * sp > sms || nkb / sp < 4)) continue;
+      const double waves = double((tiles * sp + sms - 1) / sms);
+      double t = waves * (double((nkb + sp - 1) / sp) * c.t_kb + 3.0);
+      const double part = double(tiles * sp) * c.bmt * c.bn * 4.0;
+      if (sp > 1) t += 2.0 * part / 5.0e6 + 2.0;
+      if (best.tiles == 0 || t < best_t) {  // ties keep the earlier (larger-tile, unsplit) plan
+        best_t = t;
+        best.bmt = c.bmt;
+        best.bn = c.bn;
+        best.tiles = tiles;
+        best.splitk = int(sp);
+        best.part_bytes = sp > 1 ? align256(size_t(part)) : 0;
+      }
+    }
   }
-  p.splitk = int(s);
-  p.part_bytes = s > 1 ? align256(size_t(p.tiles) * size_t(s) * size_t(p.bmt) * size_t(p.bn) * 4) : 0;
-  p.ws_bytes = s > 1 ? p.part_bytes + align256(size_t(p.tiles) * 4) : 0;
-  return p;
+  best.ws_bytes = best.part_bytes;
+  return best;
 }
 
-// Tile of the quantized GEMM.  A 256-row CTA (two accumulators sharing each
-// dequantized W tile) does twice the flops of a 128-row one for the same
-// dequantization, so one wave of them is never slower than two waves of
-// 128-row tiles: use it while it still covers about two thirds of the SMs,
-// with the widest W tile that does; else 128 rows.  Few tiles (under half the
-// SMs) split K over several CTAs per tile when the caller's workspace holds
-// the partials.
+// The quantized GEMM with the plan's tile: a 256-row CTA shares each
+// dequantized W tile between two accumulators (half the dequantization per
+// flop), a 256-wide W tile shares each X tile; the plan splits K when the
+// caller's workspace holds the partials, else it takes the best unsplit tile.
 template <int FMT>
 int launch_gemm(wq::GemmArgs& a, const uint16_t* X, const void* packed, cudaStream_t st, void* ws = nullptr,
                 size_t ws_bytes = 0) {
-  const GemmPlan p = gemm_plan(a.M, a.N, a.K);
+  GemmPlan p = gemm_plan(a.M, a.N, a.K);
   a.splitk = 1;
-  if (p.splitk > 1 && ws && ws_bytes >= p.ws_bytes && aligned16(ws)) {
+  if (p.splitk > 1 && !(ws && ws_bytes >= p.ws_bytes && aligned16(ws))) p = gemm_plan(a.M, a.N, a.K, false);
+  if (p.splitk > 1) {
     a.splitk = p.splitk;
     a.part = static_cast<float*>(ws);
-    a.ctr = reinterpret_cast<unsigned*>(static_cast<uint8_t*>(ws) + p.part_bytes);
-    // the kernel leaves the counters at 0, but the workspace may be fresh memory
-    if (int e = cuda_check(cudaMemsetAsync(a.ctr, 0, size_t(p.tiles) * 4, st), "split-K counters")) return e;
+    // the partial tiles as one fp32 matrix [tiles * splitk * BMT, BN] for the TMA stores
+    if (int e = make_tmap_2d(&a.tmPart, a.part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                             uint64_t(p.tiles) * uint64_t(p.splitk) * uint64_t(p.bmt), uint64_t(p.bn), 32, 32,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+      return e;
   }
-  if (p.bmt == 256) {
-    if (p.bn == 256) return launch_gemm_bn<FMT, 256, 256>(a, X, packed, st);
-    return launch_gemm_bn<FMT, 128, 256>(a, X, packed, st);
-  }
-  if (p.bn == 256) return launch_gemm_bn<FMT, 256>(a, X, packed, st);
-  return launch_gemm_bn<FMT, 128>(a, X, packed, st);
+  int e = WQ_OK;
+  if (p.bmt == 256)
+    e = p.bn == 256 ? launch_gemm_bn<FMT, 256, 256>(a, X, packed, st) : launch_gemm_bn<FMT, 128, 256>(a, X, packed, st);
+  else
+    e = p.bn == 256 ? launch_gemm_bn<FMT, 256>(a, X, packed, st) : launch_gemm_bn<FMT, 128>(a, X, packed, st);
+  if (e || a.splitk <= 1) return e;
+  // the split partials' sum, in split order, as a stream-ordered successor
+  const int64_t quads = p.tiles * int64_t(p.bmt) * p.bn / 4;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(std::min<int64_t>((quads + 255) / 256, 148 * 8)), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const int n_tiles = int((a.N + p.bn - 1) / p.bn);
+  return cuda_check(cudaLaunchKernelEx(&cfg, wq::split_reduce_kernel, static_cast<const float*>(a.part), a.splitk,
+                                       p.bmt, p.bn, n_tiles, quads, a.M, a.N,
+                                       FMT == wq::GEMM_NVFP4 ? a.gscale : static_cast<const float*>(nullptr), a.Y),
+                    "split reduce launch");
 }
 
 int gemm_bn(int64_t M, int64_t N) {
