@@ -994,13 +994,25 @@ def run_case(name: str):
         wq.wq_gptq_int4(W, U, 128, 1)
     elif name == "factor":
         wq.wq_gptq_hessian_factor(synth.activations_student_t(512, 11008, seed=5, device=dev))
-    elif name in ("gemm_int4", "gemm_nvfp4"):
+    elif name in ("gemm_int4", "gemm_nvfp4", "w4a4"):
         K, N, M = 2048, 11008, 2048
         W = synth.weight(N, K, seed=6, device=dev)
         X = synth.activations(M, K, seed=6, device=dev)
         p = wq.wq_quantize_int4(W, 64, 1) if name == "gemm_int4" else wq.wq_quantize_nvfp4(W)
         for _ in range(2):
-            wq.wq_linear_int4(X, p) if name == "gemm_int4" else wq.wq_linear_nvfp4(X, p)
+            if name == "gemm_int4":
+                wq.wq_linear_int4(X, p)
+            else:
+                wq.wq_linear_nvfp4(X, p, act_fp4=1 if name == "w4a4" else 0)
+    elif name == "w4a4_block":  # the W4A4 linears of one block at M = 8192 (launch lists)
+        M = 8192
+        for name_, K, N in synth.PROJECTIONS:
+            p = wq.wq_quantize_nvfp4(synth.weight(N, K, seed=7, device=dev))
+            X = synth.activations(M, K, seed=7, device=dev)
+            ws = torch.empty(wq.linear_workspace_size(M, N, K, wq.WQ_FMT_NVFP4, 1), dtype=torch.uint8, device=dev)
+            for _ in range(2):
+                wq.wq_linear_nvfp4(X, p, act_fp4=1, ws=ws)
+            del p, X, ws
     else:
         raise SystemExit(f"unknown case {name}")
     torch.cuda.synchronize()
@@ -1018,7 +1030,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-aux", action="store_true", help="skip the quantize and AWQ measurements")
     ap.add_argument("--case", help="run one small kernel case for a profiler capture and exit "
-                                   "(quant, nvfp4, proxy, awqgemm, gptq, factor, gemm_int4, gemm_nvfp4)")
+                                   "(quant, nvfp4, proxy, awqgemm, gptq, factor, gemm_int4, gemm_nvfp4, w4a4, w4a4_block)")
     args = ap.parse_args()
     if args.case:
         run_case(args.case)

@@ -169,30 +169,65 @@ __device__ __forceinline__ void load_flat8(const uint16_t* __restrict__ A, const
 }
 
 // ------------------------------------------------------------------ NVFP4
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // Pass 1: amax over the tensor, atomically max-ed into *amax_out (which the
-// host zeroed).  Non-negative floats order like their bit patterns.
+// host zeroed).  Non-negative floats order like their bit patterns.  Without
+// an AWQ scale the magnitudes are the bf16 bit patterns with the sign cleared,
+// compared as unsigned 16-bit pairs (one SIMD max per two elements, eight
+// 16-byte loads in flight per thread); a thread that saw a NaN pattern
+// (above 0x7F80) redoes its elements with fmaxf, which skips NaNs.
 __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const uint16_t* __restrict__ A, const float* __restrict__ s,
                                                          int64_t R, int64_t C, float* amax_out) {
   const int64_t words = R * C / 8;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  const int64_t t0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   float m = 0.f;
-  // four independent 16-byte loads in flight per thread per iteration
-  for (int64_t u0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u0 < words; u0 += 4 * stride) {
-    float w[4][8];
+  bool fp32_path = s != nullptr;
+  if (!fp32_path) {
+    uint32_t mi = 0;
+    for (int64_t u0 = t0; u0 < words; u0 += 8 * stride) {
+      uint4 v[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int64_t u = u0 + q * stride;
-      if (u < words) {
-        load_flat8(A, s, C, u * 8, w[q]);
-      } else {
+      for (int q = 0; q < 8; ++q) {
+        const int64_t u = u0 + q * stride;
+        v[q] = u < words ? ldg_stream_v4(A + u * 8) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) w[q][j] = 0.f;
+      for (int q = 0; q < 8; ++q) {
+        mi = max_u16x2(mi, v[q].x & 0x7FFF7FFFu);
+        mi = max_u16x2(mi, v[q].y & 0x7FFF7FFFu);
+        mi = max_u16x2(mi, v[q].z & 0x7FFF7FFFu);
+        mi = max_u16x2(mi, v[q].w & 0x7FFF7FFFu);
       }
     }
+    const uint32_t top = max(mi & 0xFFFFu, mi >> 16);
+    if (top > 0x7F80u) fp32_path = true;  // a NaN: take the fmaxf pass below for this thread
+    else m = __uint_as_float(top << 16);
+  }
+  if (fp32_path) {
+    // four independent 16-byte loads in flight per thread per iteration
+    for (int64_t u0 = t0; u0 < words; u0 += 4 * stride) {
+      float w[4][8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < 4; ++q) {
+        const int64_t u = u0 + q * stride;
+        if (u < words) {
+          load_flat8(A, s, C, u * 8, w[q]);
+        } else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(w[q][j]));
+          for (int j = 0; j < 8; ++j) w[q][j] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(w[q][j]));
+    }
   }
 #pragma unroll
   for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
@@ -231,9 +266,11 @@ __device__ __forceinline__ float nvfp4_global_from_amax(float amax) {
 // block-scale bytes and 8-byte code groups are written coalesced.
 __global__ void __launch_bounds__(256) nvfp4_pack_kernel(const uint16_t* __restrict__ A, const float* __restrict__ s,
                                                          int64_t R, int64_t C, const float* __restrict__ amax_in,
-                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ bscale) {
+                                                         uint8_t* __restrict__ codes, uint8_t* __restrict__ bscale,
+                                                         float* __restrict__ g_out) {
   const int64_t nblk = R * C / 16;
   const float g = nvfp4_global_from_amax(*amax_in);
+  if (g_out && blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;  // amax lives elsewhere: no finalize pass
   for (int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; b < nblk; b += int64_t(gridDim.x) * blockDim.x) {
     float w[16];
     load_flat8(A, s, C, b * 16, w);
