@@ -270,6 +270,8 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(const uint16_t* __restr
                                                          float* __restrict__ g_out) {
   const int64_t nblk = R * C / 16;
   const float g = nvfp4_global_from_amax(*amax_in);
+  const float rg = __frcp_rn(g);
+  const bool rg_ok = __float_as_uint(rg) < 0x7F800000u;  // not for a subnormal g (amax below ~3e-35)
   if (g_out && blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;  // amax lives elsewhere: no finalize pass
   for (int64_t b = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; b < nblk; b += int64_t(gridDim.x) * blockDim.x) {
     float w[16];
@@ -278,33 +280,44 @@ __global__ void __launch_bounds__(256) nvfp4_pack_kernel(const uint16_t* __restr
     float ab = 0.f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) ab = fmaxf(ab, fabsf(w[j]));
-    const float t = __fdiv_rn(__fdiv_rn(ab, 6.0f), g);
-    const uint32_t sb = e4m3_rn_sat(t);
+    // E4M3 block scale of the IEEE quotient (ab / 6) / g.  t = ab * fp32(1/6) *
+    // fp32(1/g) is within ~6 2^-24 (relative) of it, so the product by 1 - 2^-19
+    // and by 1 + 2^-19 bracket the quotient: when both convert to the same code
+    // (conversion is monotonic) that is its code; else the divisions are taken.
+    // The bracket needs normal intermediates: blocks with ab < 2^-120 (zero blocks
+    // among them) and a g whose reciprocal overflows take the divisions.
+    uint32_t sb;
+    {
+      const float t = __fmul_rn(__fmul_rn(ab, 1.0f / 6.0f), rg);
+      const uint32_t sl = e4m3_rn_sat(__fmul_rn(t, 1.0f - 0x1p-19f)), sh = e4m3_rn_sat(__fmul_rn(t, 1.0f + 0x1p-19f));
+      sb = sl;
+      if (__builtin_expect(sl != sh || !(ab >= 0x1p-120f) || !rg_ok, 0))
+        sb = e4m3_rn_sat(__fdiv_rn(__fdiv_rn(ab, 6.0f), g));
+    }
     const float d = e4m3_decode_pos(sb);
     uint32_t lo = 0, hi = 0;
     if (d != 0.0f) {
       const float denom = __fmul_rn(d, g);
       const float rcp = __frcp_rn(denom);
-      // Codes of the IEEE quotients w / denom, two per conversion.  t = w * rcp is
-      // within 2^-22 (relative) of the quotient; when t * (1 - 2^-19) and
-      // t * (1 + 2^-19) convert to the same pair of codes as t, every value
-      // between them does (rounding is monotonic), the quotient included.  Only
-      // pairs near a rounding boundary take the divisions.  A denominator below
+      // Codes of the IEEE quotients w / denom, two per conversion.  w * rcp is
+      // within 2^-22 (relative) of the quotient, so w * (rcp (1 - 2^-19)) and
+      // w * (rcp (1 + 2^-19)) bracket it: when they convert to the same pair of
+      // codes, so does every value between them (rounding is monotonic), the
+      // quotient included.  Only pairs near a rounding boundary take the
+      // divisions, flagged and converted in a branch of their own (rare), so the
+      // divisions are not issued, predicated off, for all.  A denominator below
       // 2^-128 (tensors with amax under ~1e-33) has no finite reciprocal: then
       // every pair takes the divisions.
-      // Pairs that take the divisions are flagged and converted in a branch of
-      // their own (rare), so the divisions are not issued, predicated off, for all.
-      const bool rcp_ok = __float_as_uint(rcp) < 0x7F800000u;
+      const float rlo = __fmul_rn(rcp, 1.0f - 0x1p-19f), rhi = __fmul_rn(rcp, 1.0f + 0x1p-19f);
+      const bool rcp_ok = __float_as_uint(rhi) < 0x7F800000u;
       uint32_t pairs[8];
       uint32_t slow = 0;
 #pragma unroll
       for (int j = 0; j < 16; j += 2) {
-        const float t0 = __fmul_rn(w[j], rcp), t1 = __fmul_rn(w[j + 1], rcp);
-        const uint32_t c = e2m1x2_rn_sat(t0, t1);
-        const uint32_t cl = e2m1x2_rn_sat(__fmul_rn(t0, 1.0f - 0x1p-19f), __fmul_rn(t1, 1.0f - 0x1p-19f));
-        const uint32_t ch = e2m1x2_rn_sat(__fmul_rn(t0, 1.0f + 0x1p-19f), __fmul_rn(t1, 1.0f + 0x1p-19f));
-        pairs[j >> 1] = c;
-        if (!(rcp_ok && c == cl && c == ch)) slow |= 1u << (j >> 1);
+        const uint32_t cl = e2m1x2_rn_sat(__fmul_rn(w[j], rlo), __fmul_rn(w[j + 1], rlo));
+        const uint32_t ch = e2m1x2_rn_sat(__fmul_rn(w[j], rhi), __fmul_rn(w[j + 1], rhi));
+        pairs[j >> 1] = cl;
+        if (!(rcp_ok && cl == ch)) slow |= 1u << (j >> 1);
       }
       if (__builtin_expect(slow != 0, 0)) {
 #pragma unroll

@@ -290,9 +290,10 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // 64-deep k-block (set by its dequantization and MMA work: 0.60 us for 128 x 128,
 // 0.80 for 256 x 128, 0.85 for 128 x 256 and 256 x 256 with every SM busy)
 // plus ~3 us to start and drain; CTAs beyond one wave of 148 queue; a split adds
-// the partial tiles' HBM round trip (~5 TB/s) and a ~2 us launch.  Splits stay
-// within one wave and keep at least 4 k-blocks per CTA.  Without a workspace
-// (allow_split false) the best unsplit plan is taken.
+// the partial tiles' round trip (~10 TB/s while they fit in L2, ~5 TB/s beyond)
+// and ~3.5 us for the reduction launch.  Splits stay within one wave and keep at
+// least 4 k-blocks per CTA.  Without a workspace (allow_split false) the best
+// unsplit plan is taken.
 struct GemmPlan {
   int bn, bmt, splitk;
   int64_t tiles;
@@ -315,7 +316,8 @@ GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K, bool allow_split = true) {
       const double waves = double((tiles * sp + sms - 1) / sms);
       double t = waves * (double((nkb + sp - 1) / sp) * c.t_kb + 3.0);
       const double part = double(tiles * sp) * c.bmt * c.bn * 4.0;
-      if (sp > 1) t += 2.0 * part / 5.0e6 + 2.0;
+      // the partials' write and read: ~10 TB/s while they fit in L2 (24 MB), ~5 TB/s past it
+      if (sp > 1) t += 2.0 * part / (part <= 24.0 * 1048576.0 ? 10.0e6 : 5.0e6) + 3.5;
       if (best.tiles == 0 || t < best_t) {  // ties keep the earlier (larger-tile, unsplit) plan
         best_t = t;
         best.bmt = c.bmt;
