@@ -80,7 +80,15 @@ __global__ void __launch_bounds__(kQuantThreads) awq_delta_kernel(const uint16_t
   }
   float sc;
   group_scale_f16(__fsub_rn(mx, mn), 15.0f, &sc);
-  const float z = fminf(fmaxf(rintf(__fdiv_rn(-mn, sc)), 0.0f), 15.0f);
+  // z = rint(-mn / sc) and q = rint(w' / sc) as the quantizer takes them: through the
+  // reciprocal, with the IEEE division (in a branch of its own) where the product
+  // lies within 2^-21 |t| of a half-integer
+  const float rsc = __frcp_rn(sc);
+  const float tz = __fmul_rn(-mn, rsc);
+  float zr = rintf(tz);
+  if (__builtin_expect(__fsub_rn(0.5f, fabsf(__fsub_rn(tz, zr))) <= fabsf(tz) * 0x1p-21f, 0))
+    zr = rintf(__fdiv_rn(-mn, sc));
+  const float z = fminf(fmaxf(zr, 0.0f), 15.0f);
   double sq = 0.0;
   if (active) {
     float sv[8];
@@ -90,12 +98,27 @@ __global__ void __launch_bounds__(kQuantThreads) awq_delta_kernel(const uint16_t
       sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
       sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
     }
+    float qr[8];
+    uint32_t slow = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float t = __fmul_rn(wp[j], rsc);
+      qr[j] = rintf(t);
+      if (__fsub_rn(0.5f, fabsf(__fsub_rn(t, qr[j]))) <= fabsf(t) * 0x1p-21f) slow |= 1u << j;
+    }
+    if (__builtin_expect(slow != 0, 0)) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (slow & (1u << j)) qr[j] = rintf(__fdiv_rn(wp[j], sc));
+    }
     uint32_t hi[4], lo[4];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float q = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(wp[j], sc)), z), 0.0f), 15.0f);
-      const float deq = __fmul_rn(__fsub_rn(q, z), sc);        // exact: |q - z| <= 15, sc has 11 bits
-      const float dl = __fsub_rn(w[j], __fdiv_rn(deq, sv[j]));  // W - dequant / s
+      const float q = fminf(fmaxf(__fadd_rn(qr[j], z), 0.0f), 15.0f);
+      const float deq = __fmul_rn(__fsub_rn(q, z), sc);  // exact: |q - z| <= 15, sc has 11 bits
+      // W - dequant / s, the quotient through the correctly rounded reciprocal of s
+      // (within an ulp of the division; Delta then travels as a bf16 hi + lo pair)
+      const float dl = __fsub_rn(w[j], __fmul_rn(deq, __frcp_rn(sv[j])));
       if (D) {
         const uint32_t h = f32_to_bf16_bits(dl);
         const uint32_t l = f32_to_bf16_bits(__fsub_rn(dl, bf16_bits_to_f32(h)));
