@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(kQuantThreads) awq_delta_kernel(const uint16_t
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   }
   float sc;
-  group_scale_f16(__fsub_rn(mx, mn), 15.0f, &sc);
+  group_scale_f16_fast(__fsub_rn(mx, mn), 15.0f, 1.0f / 15.0f, &sc);
   // z = rint(-mn / sc) and q = rint(w' / sc) as the quantizer takes them: through the
   // reciprocal, with the IEEE division (in a branch of its own) where the product
   // lies within 2^-21 |t| of a half-integer
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kAwqProxyThreads) awq_proxy_kernel(const uint1
       }
       if (!rin[r]) continue;  // whole groups share rin (a group never straddles rows or K)
       float sc;
-      group_scale_f16(__fsub_rn(mx, mn), 15.0f, &sc);
+      group_scale_f16_fast(__fsub_rn(mx, mn), 15.0f, 1.0f / 15.0f, &sc);
       const float rsc = __frcp_rn(sc);
       // z = rint(-mn / sc) and q = rint(wp / sc) through the reciprocal: |t - x / sc|
       // <= ~2^-22 |t| with |t| <= ~16, so rint(t) is the quotient's rint unless t lies

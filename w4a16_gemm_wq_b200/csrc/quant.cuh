@@ -52,6 +52,34 @@ __device__ __forceinline__ uint16_t group_scale_f16(float r, float levels, float
   return __half_as_ushort(h);
 }
 
+// The same fp16 scale without the division where it is not needed: t = r *
+// fp32(1 / levels) is within 2^-23 (relative) of the fp32 quotient, and the
+// clamp-then-round map is monotonic, so when t (1 - 2^-19) and t (1 + 2^-19)
+// map to the same fp16 that is the quotient's; otherwise (rare) the division.
+__device__ __forceinline__ uint16_t group_scale_f16_fast(float r, float levels, float rlevels, float* sc) {
+  const auto map = [](float x) {
+    if (!(x >= 1e-5f)) x = 1e-5f;
+    if (x > 65504.0f) x = 65504.0f;
+    return __half_as_ushort(__float2half_rn(x));
+  };
+  const float t = __fmul_rn(r, rlevels);
+  const uint16_t lo = map(__fmul_rn(t, 1.0f - 0x1p-19f)), hi = map(__fmul_rn(t, 1.0f + 0x1p-19f));
+  if (__builtin_expect(lo != hi, 0)) return group_scale_f16(r, levels, sc);
+  *sc = __half2float(__ushort_as_half(lo));
+  return lo;
+}
+
+// rint(x / sc) through the correctly rounded reciprocal rsc = 1 / sc: the product
+// is within 2^-23 (relative) of the IEEE quotient, so its rint is the quotient's
+// unless it lies within 2^-21 of a half-integer (relative), where the division
+// is taken (a branch of its own: rare).
+__device__ __forceinline__ float rint_quotient(float x, float sc, float rsc) {
+  const float t = __fmul_rn(x, rsc);
+  const float r = rintf(t);
+  if (__builtin_expect(__fsub_rn(0.5f, fabsf(__fsub_rn(t, r))) <= fabsf(t) * 0x1p-21f, 0)) return rintf(__fdiv_rn(x, sc));
+  return r;
+}
+
 // grid = (ceil(K/2048), N); thread t of CTA (c, n) owns word u = c*256 + t of
 // row n, i.e. k in [8u, 8u+8).  A group is G/8 consecutive lanes of one warp.
 template <int G, bool ASYM>
@@ -89,10 +117,10 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_int4_kernel(
   float sc, z = 0.f;
   uint16_t hbits;
   if (ASYM) {
-    hbits = group_scale_f16(__fsub_rn(mx, mn), 15.0f, &sc);
-    z = fminf(fmaxf(rintf(__fdiv_rn(-mn, sc)), 0.0f), 15.0f);
+    hbits = group_scale_f16_fast(__fsub_rn(mx, mn), 15.0f, 1.0f / 15.0f, &sc);
+    z = fminf(fmaxf(rint_quotient(-mn, sc, __frcp_rn(sc)), 0.0f), 15.0f);
   } else {
-    hbits = group_scale_f16(amax, 7.0f, &sc);
+    hbits = group_scale_f16_fast(amax, 7.0f, 1.0f / 7.0f, &sc);
   }
   if (active) {
     uint32_t word = 0;
