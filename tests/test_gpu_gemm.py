@@ -42,8 +42,9 @@ def test_small_gemm_all_rows(lib, M, fmt):
     assert_linear_close(Y, ref, what=f"{fmt} M={M}")
 
 
-@pytest.mark.parametrize("K,N", [(96, 40), (1056, 200), (2048, 520)])
+@pytest.mark.parametrize("K,N", [(96, 40), (1056, 200), (2048, 520), (2048, 203)])
 def test_ragged_k_and_n(lib, K, N):
+    # N % 8 != 0 (203) stores Y row by row instead of by TMA boxes
     M = 160
     W = synth.weight(N, K, seed=K)
     X = synth.activations(M, K, seed=N)
@@ -121,12 +122,14 @@ def test_two_accumulator_tiles_ragged(lib, M, N, fmt):
 
 
 @pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
-@pytest.mark.parametrize("M,N,K", [(512, 256, 11008), (2048, 256, 4096), (512, 2048, 11008), (300, 200, 3072)])
+@pytest.mark.parametrize("M,N,K", [(512, 256, 11008), (2048, 256, 4096), (512, 2048, 11008), (300, 200, 3072),
+                                   (512, 203, 11008)])
 def test_split_k_few_tiles(lib, fmt, M, N, K):
     # few output tiles: K split over several CTAs per tile through the workspace
-    # (fp32 partials, the last CTA of a tile sums them in split order): sampled rows
-    # against the oracle, bit-identical on a second run with the same workspace (the
-    # counters start as garbage and must come back to 0), and close to the unsplit run
+    # (fp32 partial tiles by TMA, then the reduction launch sums them in split
+    # order): sampled rows against the oracle, bit-identical on a second run with the
+    # same (garbage-filled) workspace, and close to the unsplit run; N = 203 takes the
+    # reduction's element-wise Y stores
     W = synth.weight(N, K, seed=M + N + K, device="cuda")
     X = synth.activations(M, K, seed=K, device="cuda")
     p = lib.wq_quantize_int4(W, 64, 1) if fmt == "int4" else lib.wq_quantize_nvfp4(W)

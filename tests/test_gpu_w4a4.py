@@ -36,8 +36,9 @@ def _run(lib, X, p, inv_s=None):
 
 
 @pytest.mark.parametrize("M", [1, 17, 128, 200])
-@pytest.mark.parametrize("K,N", [(64, 40), (320, 256), (2048, 384)])
+@pytest.mark.parametrize("K,N", [(64, 40), (320, 256), (2048, 384), (2048, 203)])
 def test_w4a4_small(lib, M, K, N):
+    # N = 203 (N % 8 != 0) stores Y row by row instead of by TMA boxes
     W = synth.weight(N, K, seed=K + N)
     X = synth.activations(M, K, seed=M + K, channels=synth.outlier_channels(K, 0.01, 1))
     p = lib.wq_quantize_nvfp4(W.cuda())
