@@ -437,7 +437,12 @@ __global__ void __launch_bounds__(Fp4PShape::THREADS, 1) gemm_fp4_persistent_ker
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC = idesc_nvf4(kGemmBM, BN);
-      int q = 0, i = 0;
+      // stage 0's operand descriptors and scale columns; stage s adds s stages (the
+      // descriptor's start address is addr / 16 in its low 14 bits: no carry below 256 KB)
+      const uint64_t ad0 = desc_kmajor_sw128(sbase), bd0 = desc_kmajor_sw128(sbase + uint32_t(S::A_BYTES));
+      const uint32_t sfa0 = tmem + sfa_col(0), sfb0 = tmem + sfb_col(0);
+      int q = 0, i = 0, s = 0;
+      uint32_t par = 0;  // phase parity of stage s's barriers
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++i) {
         const int b = i & 1, u = i >> 1;
@@ -445,20 +450,24 @@ __global__ void __launch_bounds__(Fp4PShape::THREADS, 1) gemm_fp4_persistent_ker
         tc_fence_after();
         const uint32_t dacc = tmem + uint32_t(b * BN);
         for (int kb = 0; kb < nkb; ++kb, ++q) {
-          const int s = q % STAGES, r = q / STAGES;
-          if (!mbar_wait(&full[s], r & 1, ERR_TIMEOUT_TMA, abort_flag) ||
-              !mbar_wait(&sfready[s], r & 1, ERR_TIMEOUT_PIPE, abort_flag)) {
+          if (!mbar_wait(&full[s], par, ERR_TIMEOUT_TMA, abort_flag) ||
+              !mbar_wait(&sfready[s], par, ERR_TIMEOUT_PIPE, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t ad = desc_kmajor_sw128(sbase + uint32_t(s * S::STAGE_BYTES));
-          const uint64_t bd = desc_kmajor_sw128(sbase + uint32_t(s * S::STAGE_BYTES + S::A_BYTES));
+          const uint64_t ad = ad0 + uint64_t(s * (S::STAGE_BYTES >> 4));
+          const uint64_t bd = bd0 + uint64_t(s * (S::STAGE_BYTES >> 4));
+          const uint32_t sfa = sfa0 + uint32_t(s * S::SF_STAGE_COLS), sfb = sfb0 + uint32_t(s * S::SF_STAGE_COLS);
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4)
-            umma_nvf4(dacc, ad + uint64_t(2 * k4), bd + uint64_t(2 * k4), IDESC, tmem + sfa_col(s) + 4 * k4,
-                      tmem + sfb_col(s) + 4 * k4, (kb | k4) != 0);
+            umma_nvf4(dacc, ad + uint64_t(2 * k4), bd + uint64_t(2 * k4), IDESC, sfa + 4 * k4, sfb + 4 * k4,
+                      (kb | k4) != 0);
           umma_commit(&empty[s]);
+          if (++s == STAGES) {
+            s = 0;
+            par ^= 1u;
+          }
         }
         umma_commit(&acc_full[b]);  // also after an abort: completes when the issued MMAs are done
       }
