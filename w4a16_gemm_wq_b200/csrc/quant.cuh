@@ -210,7 +210,8 @@ __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
 // 16-byte loads in flight per thread); a thread that saw a NaN pattern
 // (above 0x7F80) redoes its elements with fmaxf, which skips NaNs.
 __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const uint16_t* __restrict__ A, const float* __restrict__ s,
-                                                         int64_t R, int64_t C, float* amax_out) {
+                                                         int64_t R, int64_t C, float* amax_out,
+                                                         float* __restrict__ block_max) {
   const int64_t words = R * C / 8;
   const int64_t stride = int64_t(gridDim.x) * blockDim.x;
   const int64_t t0 = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -264,8 +265,25 @@ __global__ void __launch_bounds__(256) nvfp4_amax_kernel(const uint16_t* __restr
   __syncthreads();
   if (threadIdx.x == 0) {
     for (int i = 1; i < int(blockDim.x >> 5); ++i) m = fmaxf(m, red[i]);
-    atomicMax(reinterpret_cast<unsigned int*>(amax_out), __float_as_uint(m));
+    if (block_max)
+      block_max[blockIdx.x] = m;  // the pack pass takes the maximum of these (no zeroing, no atomics)
+    else
+      atomicMax(reinterpret_cast<unsigned int*>(amax_out), __float_as_uint(m));
   }
+}
+
+// amax from the amax pass's per-CTA maxima (n of them), the same value in every thread
+__device__ __forceinline__ float nvfp4_amax_of_blocks(const float* __restrict__ block_max, int n) {
+  __shared__ float red[8];
+  float m = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, block_max[i]);
+#pragma unroll
+  for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  m = red[0];
+  for (int i = 1; i < int(blockDim.x >> 5); ++i) m = fmaxf(m, red[i]);
+  return m;
 }
 
 // Hardware conversions: round to nearest with ties to the even mantissa (for
@@ -295,9 +313,11 @@ __device__ __forceinline__ float nvfp4_global_from_amax(float amax) {
 __global__ void __launch_bounds__(256) nvfp4_pack_kernel(const uint16_t* __restrict__ A, const float* __restrict__ s,
                                                          int64_t R, int64_t C, const float* __restrict__ amax_in,
                                                          uint8_t* __restrict__ codes, uint8_t* __restrict__ bscale,
-                                                         float* __restrict__ g_out) {
+                                                         float* __restrict__ g_out, const float* __restrict__ block_max,
+                                                         int n_block_max) {
   const int64_t nblk = R * C / 16;
-  const float g = nvfp4_global_from_amax(*amax_in);
+  // the tensor's amax: accumulated by the amax pass, or its per-CTA maxima reduced here
+  const float g = nvfp4_global_from_amax(block_max ? nvfp4_amax_of_blocks(block_max, n_block_max) : *amax_in);
   const float rg = __frcp_rn(g);
   const bool rg_ok = __float_as_uint(rg) < 0x7F800000u;  // not for a subnormal g (amax below ~3e-35)
   if (g_out && blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;  // amax lives elsewhere: no finalize pass

@@ -425,13 +425,14 @@ struct W4A4Layout {
   size_t off_codes, off_sf, off_g, total;
 };
 
-constexpr int kW4A4AmaxSlot = 32;  // floats past g_x: the activation amax accumulator (same 256-byte slot)
+// The activation amax pass's per-CTA maxima follow g_x's 256-byte slot.
+constexpr int kW4A4AmaxSlot = 64;  // floats past g_x
 W4A4Layout w4a4_layout(int64_t M, int64_t K) {
   W4A4Layout L = {};
   L.off_codes = 0;
   L.off_sf = align256(size_t(M) * size_t(K / 2));
   L.off_g = align256(L.off_sf + size_t(M) * size_t(K / 16));
-  L.total = L.off_g + 256;
+  L.total = L.off_g + 256 + align256(size_t(4 * 148 * 8));
   return L;
 }
 
@@ -508,22 +509,25 @@ int launch_fp4_bn(wq::Fp4Args& a, const uint8_t* xcodes, const uint8_t* wcodes, 
 
 // NVFP4 quantization of a bf16 [R, C] tensor (optionally times s per column)
 // into codes / scales / g: the stream-ordered passes of wq_quantize_nvfp4
-// (amax, pack, and a one-thread pass that turns the amax in *g into g).  With
-// amax_scratch (a float the caller does not otherwise use) the amax goes there
-// and the pack pass writes g itself, one launch fewer.
+// (zeroing, an atomic amax pass, pack, and a one-thread pass that turns the
+// amax in *g into g).  With block_max scratch (kNvfp4AmaxBlocks floats the caller
+// does not otherwise use) the amax pass leaves one maximum per CTA there and the
+// pack pass reduces them and writes g itself: two launches fewer.
+constexpr int kNvfp4AmaxBlocks = 148 * 8;
 int nvfp4_quantize_launch(const uint16_t* A, int64_t R, int64_t C, const float* s, uint8_t* codes, uint8_t* bscale,
-                          float* g, cudaStream_t st, float* amax_scratch = nullptr) {
-  float* amax = amax_scratch ? amax_scratch : g;
-  if (int e = cuda_check(cudaMemsetAsync(amax, 0, sizeof(float), st), "memset")) return e;
+                          float* g, cudaStream_t st, float* block_max = nullptr) {
   const int64_t words = R * C / 8;
-  const int amax_blocks = int(std::min<int64_t>((words + 255) / 256, 148 * 8));
-  wq::nvfp4_amax_kernel<<<amax_blocks, 256, 0, st>>>(A, s, R, C, amax);
+  const int amax_blocks = int(std::max<int64_t>(1, std::min<int64_t>((words + 255) / 256, kNvfp4AmaxBlocks)));
+  if (!block_max)
+    if (int e = cuda_check(cudaMemsetAsync(g, 0, sizeof(float), st), "memset")) return e;
+  wq::nvfp4_amax_kernel<<<amax_blocks, 256, 0, st>>>(A, s, R, C, g, block_max);
   if (int e = launched("nvfp4_amax launch")) return e;
   const int64_t nblk = R * C / 16;
-  const int pack_blocks = int(std::min<int64_t>((nblk + 255) / 256, 148 * 16));
-  wq::nvfp4_pack_kernel<<<pack_blocks, 256, 0, st>>>(A, s, R, C, amax, codes, bscale, amax_scratch ? g : nullptr);
+  const int pack_blocks = int(std::max<int64_t>(1, std::min<int64_t>((nblk + 255) / 256, 148 * 16)));
+  wq::nvfp4_pack_kernel<<<pack_blocks, 256, 0, st>>>(A, s, R, C, g, codes, bscale, block_max ? g : nullptr,
+                                                      block_max, amax_blocks);
   if (int e = launched("nvfp4_pack launch")) return e;
-  if (amax_scratch) return WQ_OK;
+  if (block_max) return WQ_OK;
   wq::nvfp4_finalize_kernel<<<1, 1, 0, st>>>(g);
   return launched("nvfp4_finalize launch");
 }
@@ -1481,7 +1485,7 @@ int wq_linear_nvfp4_w4a4_noalloc(const uint16_t* X, int64_t M, int64_t N, int64_
   uint8_t* xcodes = wsb + L.off_codes;
   uint8_t* xsf = wsb + L.off_sf;
   float* gx = reinterpret_cast<float*>(wsb + L.off_g);
-  // nvfp4_quantize_launch zeroes the amax accumulator (beside g_x) before using it
+  // the amax pass's per-CTA maxima go after g_x's slot; the pack pass reduces them and writes g_x
   if (int e = nvfp4_quantize_launch(X, M, K, act_inv_s, xcodes, xsf, gx, st, gx + kW4A4AmaxSlot)) return e;
   wq::Fp4Args f = {};
   f.sfa = xsf; f.sfb = bscale; f.gx = gx; f.gw = global_scale; f.Y = Y;
