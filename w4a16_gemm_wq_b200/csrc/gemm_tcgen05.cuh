@@ -455,7 +455,7 @@ __global__ void __launch_bounds__(GemmShape<BN, BMT, FMT == GEMM_BF16_SQ>::THREA
     constexpr int WPQ = DEQ_WARPS / 4;                 // epilogue warps per lane quarter
     const int wi = (warp - DEQ_WARP0) >> 2;            // this warp's index among them
     const bool vec = (a.N % 8) == 0;
-    if (FMT != GEMM_BF16_SQ && a.splitk > 1) {
+    if (a.splitk > 1) {
       // split-K: this CTA's fp32 partial tile leaves by TMA (32 x 32 boxes staged in
       // the freed stage buffers, 128-byte swizzle); split_reduce_kernel, launched
       // next, adds the partials in split order and writes Y (no CTA waits for
@@ -615,6 +615,54 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(const float* __restri
       for (int q = 0; q < 4; ++q)
         if (col + q < N) yp[q] = uint16_t(f32_to_bf16_bits(tv[q] * gmul));
     }
+  }
+}
+
+// Split-K for the AWQ loss GEMM: the sum over one tile's rows ry*16 .. ry*16+15 of
+// y^2, y = the splits' partials added in split order, into partials[tile * 8 + ry]
+// (gridDim.y = 8 row slices of a 128-row tile).  Each thread takes float4 column
+// groups of those rows with every split's load in flight; fixed-order reductions.
+__global__ void __launch_bounds__(256) split_sq_reduce_kernel(const float* __restrict__ part, int splitk, int bn,
+                                                              int n_tiles, int M, int N, double* __restrict__ partials) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int tile = blockIdx.x, ry = blockIdx.y;
+  const int m0 = (tile / n_tiles) * kGemmBM, n0 = (tile % n_tiles) * bn;
+  const int64_t tile_elems = int64_t(kGemmBM) * bn;
+  const float* base = part + int64_t(tile) * splitk * tile_elems;
+  const int quads = 16 * bn / 4;
+  double sq = 0.0;
+  for (int qd = threadIdx.x; qd < quads; qd += blockDim.x) {
+    const int rt = ry * 16 + (qd * 4) / bn, ct = (qd * 4) % bn;
+    const float4* src = reinterpret_cast<const float4*>(base + int64_t(rt) * bn + ct);
+    float4 x[8];
+#pragma unroll
+    for (int sp = 0; sp < 8; ++sp)
+      if (sp < splitk) x[sp] = __ldcs(src + sp * (tile_elems / 4));
+    float4 t = x[0];
+#pragma unroll
+    for (int sp = 1; sp < 8; ++sp)
+      if (sp < splitk) {
+        t.x += x[sp].x; t.y += x[sp].y; t.z += x[sp].z; t.w += x[sp].w;
+      }
+    const int row = m0 + rt, col = n0 + ct;
+    float acc = 0.f;
+    if (row < M) {
+      if (col < N) acc = fmaf(t.x, t.x, acc);
+      if (col + 1 < N) acc = fmaf(t.y, t.y, acc);
+      if (col + 2 < N) acc = fmaf(t.z, t.z, acc);
+      if (col + 3 < N) acc = fmaf(t.w, t.w, acc);
+    }
+    sq += double(acc);
+  }
+  __shared__ double red[8];
+#pragma unroll
+  for (int off = 16; off; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sq;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tsum = 0.0;
+    for (int w = 0; w < int(blockDim.x >> 5); ++w) tsum += red[w];
+    partials[int64_t(tile) * 8 + ry] = tsum;
   }
 }
 

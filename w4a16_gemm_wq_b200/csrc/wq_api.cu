@@ -386,6 +386,9 @@ struct AwqLayout {
   size_t off_a, off_s, off_p, off_d, total;
   int64_t P;
   int bn;
+  int splitk;          // loss GEMM: CTAs per output tile along K (1 = the fused sum-of-squares epilogue)
+  int64_t tiles;       // loss GEMM output tiles
+  size_t off_part;     // loss GEMM split partial tiles (fp32 [tiles * splitk * 128, bn])
 };
 
 // Without tokens and with at most kAwqProxyMaxAlphas alphas the search runs the
@@ -394,11 +397,20 @@ struct AwqLayout {
 bool awq_fused_proxy(bool has_x, int n_alpha) { return !has_x && n_alpha <= wq::kAwqProxyMaxAlphas; }
 int64_t awq_proxy_kx(int64_t K) { return (K / 8 + wq::kAwqProxyThreads - 1) / wq::kAwqProxyThreads; }
 
+// The loss GEMM [T, 2K] x [N, 2K]^T (K' = 2K) splits K' when its tiles leave SMs idle:
+// the split partial tiles, then kAwqSqRows reduction CTAs per tile that add them in
+// split order, square and sum (one partial slot each).
+constexpr int kAwqSqRows = 8;
 AwqLayout awq_layout(int64_t N, int64_t K, int64_t T, bool has_x, int n_alpha) {
   AwqLayout L = {};
+  L.splitk = 1;
   if (has_x) {
     L.bn = gemm_bn(T, N);
-    L.P = ((N + L.bn - 1) / L.bn) * ((T + wq::kGemmBM - 1) / wq::kGemmBM) * (L.bn / 32);
+    L.tiles = ((N + L.bn - 1) / L.bn) * ((T + wq::kGemmBM - 1) / wq::kGemmBM);
+    const int64_t nkb = 2 * K / wq::kGemmBK;
+    for (int sp = 8; sp >= 2; sp /= 2)  // the most splits that stay within one wave, >= 8 k-blocks each
+      if (L.splitk == 1 && L.tiles * sp <= wq::kTcMaxCtas && nkb / sp >= 8) L.splitk = sp;
+    L.P = L.splitk > 1 ? L.tiles * kAwqSqRows : L.tiles * (L.bn / 32);
   } else if (awq_fused_proxy(has_x, n_alpha)) {
     L.bn = 0;
     L.P = awq_proxy_kx(K) * ((N + wq::kAwqProxyRows - 1) / wq::kAwqProxyRows + 63);
@@ -410,9 +422,10 @@ AwqLayout awq_layout(int64_t N, int64_t K, int64_t T, bool has_x, int n_alpha) {
   L.off_s = align256(L.off_a + size_t(K) * 8);
   L.off_p = align256(L.off_s + size_t(K) * 4);
   L.off_d = align256(L.off_p + size_t(n_alpha) * size_t(L.P) * 8);
-  if (has_x)
-    L.total = align256(L.off_d + size_t(N) * size_t(2 * K) * 2);
-  else if (awq_fused_proxy(has_x, n_alpha))
+  if (has_x) {
+    L.off_part = align256(L.off_d + size_t(N) * size_t(2 * K) * 2);
+    L.total = L.off_part + (L.splitk > 1 ? align256(size_t(L.tiles) * L.splitk * wq::kGemmBM * L.bn * 4) : 0);
+  } else if (awq_fused_proxy(has_x, n_alpha))
     L.total = align256(L.off_d + size_t(2 * n_alpha + 1) * size_t(K) * 4);
   else
     L.total = L.off_d;
@@ -1201,6 +1214,14 @@ static int awq_search_pieces(const uint16_t* const* Ws, const int64_t* Ns, int n
     if (int e = make_tmap_2d(&g.tmP, D, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, uint64_t(N), uint64_t(2 * K), L.bn,
                              wq::kGemmBK, CU_TENSOR_MAP_SWIZZLE_128B))
       return e;
+    if (L.splitk > 1) {  // partial tiles by TMA, then the sum-of-squares reduction
+      g.splitk = L.splitk;
+      g.part = reinterpret_cast<float*>(wsb + L.off_part);
+      if (int e = make_tmap_2d(&g.tmPart, g.part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                               uint64_t(L.tiles) * uint64_t(L.splitk) * wq::kGemmBM, uint64_t(L.bn), 32, 32,
+                               CU_TENSOR_MAP_SWIZZLE_128B))
+        return e;
+    }
   }
   const unsigned gx = unsigned((K / 8 + wq::kQuantThreads - 1) / wq::kQuantThreads);
   for (int i = 0; i < n_alpha; ++i) {
@@ -1226,6 +1247,12 @@ static int awq_search_pieces(const uint16_t* const* Ws, const int64_t* Ns, int n
       const int e = (L.bn == 256) ? launch_gemm_prepared<wq::GEMM_BF16_SQ, 256>(g, st)
                                   : launch_gemm_prepared<wq::GEMM_BF16_SQ, 128>(g, st);
       if (e) return e;
+      if (L.splitk > 1) {
+        const int n_tiles = int((N + L.bn - 1) / L.bn);
+        wq::split_sq_reduce_kernel<<<dim3(unsigned(L.tiles), kAwqSqRows), 256, 0, st>>>(
+            g.part, L.splitk, L.bn, n_tiles, int(T), int(N), part_i);
+        if (int e2 = launched("awq loss reduce launch")) return e2;
+      }
     }
   }
   wq::awq_finalize_kernel<<<1, 256, 0, st>>>(partials, L.P, n_alpha, a, alphas, K, loss_out, best_idx, s_out);
