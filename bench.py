@@ -437,7 +437,8 @@ def run_ours(args):
         results = prefill_measure(wq, synth, torch, dev, peaks, rank=rank)
         out["prefill"] = {"workload": "block of 7 projections (q,k,v,o,gate,up,down) at M rows: INT4 g64 and NVFP4 "
                                       "W4A16 (gemm_tcgen05_kernel, bf16 tcgen05), NVFP4 W4A4 (activation pack + "
-                                      "gemm_fp4_kernel, block-scaled FP4 tcgen05); bf16 X ~N(0,1)",
+                                      "gemm_fp4_kernel, block-scaled FP4 tcgen05); bf16 X ~N(0,1); keys ending in _fused: "
+                                      "the same block with q/k/v and gate/up stacked along N (4 GEMMs)",
                           "peak_tflops": {"bf16_burst": peaks["bf16"], "bf16_sustained": peaks["bf16_sustained"],
                                           "fp4_burst": peaks["fp4"], "fp4_sustained": peaks["fp4_sustained"],
                                           "source": peaks["source"] + " bf16; fp4: " + peaks["fp4_source"]},
@@ -531,64 +532,72 @@ def prefill_measure(wq, synth, torch, dev, peaks, Ms=(512, 2048, 8192), reps=20,
     """Config-4 prefill: the 7 projections of one block at M rows, INT4 g64 and
     NVFP4 (W4A16), each GEMM captured in a CUDA graph of `reps` launches
     (rotating 2 weight copies) and timed with CUDA events.  Returns TFLOP/s
-    per (format, M) over the whole block and per projection."""
+    per (format, M) over the whole block and per projection; the keys ending in
+    `_fused` time the same block with q/k/v and gate/up stacked along N (4 GEMMs,
+    the same flops; W4A4 then packs each distinct input once)."""
     out = {}
     for fmt in ("int4_g64", "nvfp4", "nvfp4_w4a4"):
-        packs = []
-        for copy in range(2):
-            row = []
-            for name, K, N in synth.PROJECTIONS:
-                W = synth.weight(N, K, seed=synth.layer_seed(4, 10 * copy + K + N + 1000 * rank), device=dev)
-                row.append((name, K, N, wq.wq_quantize_int4(W, 64, 1) if fmt == "int4_g64" else wq.wq_quantize_nvfp4(W)))
-                del W
-            packs.append(row)
-        for M in Ms:
-            Xs = {K: synth.activations(M, K, seed=synth.layer_seed(4, M + K), device=dev) for _, K, _ in synth.PROJECTIONS}
-            Ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _, _, N in synth.PROJECTIONS}
-            ws = None
-            if fmt == "nvfp4_w4a4":
-                need = max(wq.linear_workspace_size(M, N, K, wq.WQ_FMT_NVFP4, 1) for _, K, N in synth.PROJECTIONS)
-                ws = torch.empty(need, dtype=torch.uint8, device=dev)
-            per = {}
-            tot_flop, tot_s = 0.0, 0.0
-            for j, (name, K, N, _) in enumerate(packs[0]):
-                def call(p, K=K, N=N):
-                    if fmt == "nvfp4":
-                        wq.wq_linear_nvfp4(Xs[K], p, out=Ys[N])
-                    elif fmt == "nvfp4_w4a4":
-                        wq.wq_linear_nvfp4(Xs[K], p, act_fp4=1, out=Ys[N], ws=ws)
-                    else:
-                        wq.wq_linear_int4(Xs[K], p, out=Ys[N])
-                call(packs[0][j][3])
-                call(packs[1][j][3])
-                torch.cuda.synchronize()
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    for r in range(reps):
-                        call(packs[r % 2][j][3])
-                g.replay()
-                torch.cuda.synchronize()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record()
-                g.replay()
-                b.record()
-                torch.cuda.synchronize()
-                sec = a.elapsed_time(b) * 1e-3 / reps
-                flop = 2.0 * M * N * K
-                per[name] = round(flop / sec / 1e12, 1)
-                tot_flop += flop
-                tot_s += sec
-                del g
-            tf = tot_flop / tot_s / 1e12
-            pk = peaks["fp4"] if fmt == "nvfp4_w4a4" else peaks["bf16"]
-            pks = peaks["fp4_sustained"] if fmt == "nvfp4_w4a4" else peaks["bf16_sustained"]
-            out[f"{fmt}_M{M}"] = {"TFLOP/s": round(tf, 1), "peak": "fp4" if fmt == "nvfp4_w4a4" else "bf16",
-                                  "frac_of_sustained": round(tf / pks, 4), "frac_of_burst": round(tf / pk, 4),
-                                  "per_projection_TFLOP/s": per, "us_per_block": round(tot_s * 1e6, 1)}
-            del Xs, Ys, ws
-        del packs
+        for layout, projs in (("", synth.PROJECTIONS), ("_fused", synth.FUSED_PROJECTIONS)):
+            _prefill_block(wq, synth, torch, dev, peaks, Ms, reps, rank, fmt, layout, projs, out)
     torch.cuda.empty_cache()
     return out
+
+
+def _prefill_block(wq, synth, torch, dev, peaks, Ms, reps, rank, fmt, layout, projs, out):
+    """One block layout of the prefill measurement for one format, at every M."""
+    packs = []
+    for copy in range(2):
+        row = []
+        for name, K, N in projs:
+            W = synth.weight(N, K, seed=synth.layer_seed(4, 10 * copy + K + N + 1000 * rank), device=dev)
+            row.append((name, K, N, wq.wq_quantize_int4(W, 64, 1) if fmt == "int4_g64" else wq.wq_quantize_nvfp4(W)))
+            del W
+        packs.append(row)
+    for M in Ms:
+        Xs = {K: synth.activations(M, K, seed=synth.layer_seed(4, M + K), device=dev) for _, K, _ in projs}
+        Ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _, _, N in projs}
+        ws = None
+        if fmt == "nvfp4_w4a4":
+            need = max(wq.linear_workspace_size(M, N, K, wq.WQ_FMT_NVFP4, 1) for _, K, N in projs)
+            ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        per = {}
+        tot_flop, tot_s = 0.0, 0.0
+        for j, (name, K, N, _) in enumerate(packs[0]):
+            def call(p, K=K, N=N):
+                if fmt == "nvfp4":
+                    wq.wq_linear_nvfp4(Xs[K], p, out=Ys[N])
+                elif fmt == "nvfp4_w4a4":
+                    wq.wq_linear_nvfp4(Xs[K], p, act_fp4=1, out=Ys[N], ws=ws)
+                else:
+                    wq.wq_linear_int4(Xs[K], p, out=Ys[N])
+            call(packs[0][j][3])
+            call(packs[1][j][3])
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for r in range(reps):
+                    call(packs[r % 2][j][3])
+            g.replay()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            torch.cuda.synchronize()
+            sec = a.elapsed_time(b) * 1e-3 / reps
+            flop = 2.0 * M * N * K
+            per[name] = round(flop / sec / 1e12, 1)
+            tot_flop += flop
+            tot_s += sec
+            del g
+        tf = tot_flop / tot_s / 1e12
+        pk = peaks["fp4"] if fmt == "nvfp4_w4a4" else peaks["bf16"]
+        pks = peaks["fp4_sustained"] if fmt == "nvfp4_w4a4" else peaks["bf16_sustained"]
+        out[f"{fmt}_M{M}{layout}"] = {"TFLOP/s": round(tf, 1), "peak": "fp4" if fmt == "nvfp4_w4a4" else "bf16",
+                                      "frac_of_sustained": round(tf / pks, 4), "frac_of_burst": round(tf / pk, 4),
+                                      "per_projection_TFLOP/s": per, "us_per_block": round(tot_s * 1e6, 1)}
+        del Xs, Ys, ws
+    del packs
 
 
 def quant_measure(wq, synth, torch, dev, peaks, reps=10):

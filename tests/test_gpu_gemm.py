@@ -78,13 +78,17 @@ def _sampled_rows(M, n=24):
     return np.array(sorted(r for r in rows if r < M))
 
 
-@pytest.mark.parametrize("name,K,N", synth.PROJECTIONS)
+# the 7 projections, and the stacked q/k/v and gate/up Linears of the fused block layout
+_BLOCK_SHAPES = list(synth.PROJECTIONS) + [p for p in synth.FUSED_PROJECTIONS if p[0] in ("qkv_proj", "gate_up_proj")]
+
+
+@pytest.mark.parametrize("name,K,N", _BLOCK_SHAPES)
 @pytest.mark.parametrize("M", [512, 2048, 8192])
 @pytest.mark.parametrize("fmt", ["int4_g64", "nvfp4"])
 def test_config4_block_projection_sampled(lib, name, K, N, M, fmt):
-    # every projection of the block at every prefill size the benchmark times, in the
-    # benchmark's launch configuration (no workspace), on sampled rows (every row band
-    # of the tiles plus the ragged tail)
+    # every Linear of the block (both layouts) at every prefill size the benchmark times,
+    # in the benchmark's launch configuration (no workspace), on sampled rows (every row
+    # band of the tiles plus the ragged tail)
     W = synth.weight(N, K, seed=synth.layer_seed(4, K + N), device="cuda")
     X = synth.activations(M, K, seed=synth.layer_seed(4, M), device="cuda")
     if fmt == "nvfp4":

@@ -64,11 +64,12 @@ def test_w4a4_with_awq_inv_scale(lib):
     assert_linear_close(Y, oracle.matmul_abT(oracle.dequant_nvfp4(ref), _wref(p)), what="w4a4 inv_s")
 
 
-@pytest.mark.parametrize("name,K,N", synth.PROJECTIONS)
+@pytest.mark.parametrize("name,K,N", list(synth.PROJECTIONS)
+                         + [p for p in synth.FUSED_PROJECTIONS if p[0] in ("qkv_proj", "gate_up_proj")])
 @pytest.mark.parametrize("M", [512, 2048, 8192])
 def test_config4_w4a4_sampled(lib, name, K, N, M):
-    # every projection at every prefill size the benchmark times: the activation pack
-    # bit-exact in full, Y on sampled rows
+    # every Linear of the block (both layouts) at every prefill size the benchmark times:
+    # the activation pack bit-exact in full, Y on sampled rows
     W = synth.weight(N, K, seed=synth.layer_seed(4, K + N), device="cuda")
     X = synth.activations(M, K, seed=synth.layer_seed(4, M), device="cuda")
     p = lib.wq_quantize_nvfp4(W)

@@ -27,6 +27,17 @@ PROJECTIONS = (
     ("down_proj", 11008, 2048),
 )
 
+# The same block as an inference engine runs it: the projections that read one
+# input stacked along N into one Linear (q/k/v after the attention norm,
+# gate/up after the MLP norm), the layout the shared-s AWQ scale serves
+# (one s per norm, folded into that norm).  Same flops as PROJECTIONS.
+FUSED_PROJECTIONS = (
+    ("qkv_proj", 2048, 2048 + 256 + 256),
+    ("o_proj", 2048, 2048),
+    ("gate_up_proj", 2048, 2 * 11008),
+    ("down_proj", 11008, 2048),
+)
+
 # The four distinct decode shapes (K, N) of the block.
 DECODE_SHAPES = ((2048, 2048), (2048, 256), (2048, 11008), (11008, 2048))
 
