@@ -132,7 +132,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_mma_kernel(const GemvMmaA
   // ---- this lane's codes and metadata of step j, kMmaDepth steps in flight
   struct Entry {
     uint4 lo, hi;
-    uint32_t mlo, mhi;  // INT4: fp16 scale | zero nibble << 16; NVFP4: the two E4M3 bytes of the lane's blocks
+    uint32_t mlo, mhi;  // INT4: fp16 scale; NVFP4: the two E4M3 bytes of the lane's blocks
+    uint32_t zlo, zhi;  // INT4: the packed zero-point words holding this step's group (decoded at use)
   };
   const auto load = [&](int j, Entry& e) {
     e.lo = tc_ld_stream(clo + 64 * j);
@@ -140,10 +141,10 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_mma_kernel(const GemvMmaA
     const int k = j * kMmaStepK + 32 * c;
     if (FMT == FMT_INT4) {
       const int grp = k >> a.log2g;
-      const uint32_t zl = a.zeros ? (__ldg(a.zeros + int64_t(nlo) * zw + (grp >> 3)) >> (4 * (grp & 7))) & 0xFu : 8u;
-      const uint32_t zh = a.zeros ? (__ldg(a.zeros + int64_t(nhi) * zw + (grp >> 3)) >> (4 * (grp & 7))) & 0xFu : 8u;
-      e.mlo = uint32_t(__ldg(a.scales + int64_t(nlo) * ng + grp)) | (zl << 16);
-      e.mhi = uint32_t(__ldg(a.scales + int64_t(nhi) * ng + grp)) | (zh << 16);
+      e.zlo = a.zeros ? __ldg(a.zeros + int64_t(nlo) * zw + (grp >> 3)) : 0x88888888u;
+      e.zhi = a.zeros ? __ldg(a.zeros + int64_t(nhi) * zw + (grp >> 3)) : 0x88888888u;
+      e.mlo = __ldg(a.scales + int64_t(nlo) * ng + grp);
+      e.mhi = __ldg(a.scales + int64_t(nhi) * ng + grp);
     } else {
       e.mlo = __ldg(reinterpret_cast<const uint16_t*>(a.bscale + int64_t(nlo) * (K >> 4) + (k >> 4)));
       e.mhi = __ldg(reinterpret_cast<const uint16_t*>(a.bscale + int64_t(nhi) * (K >> 4) + (k >> 4)));
@@ -215,7 +216,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_mma_kernel(const GemvMmaA
         const float fl = __half2float(__ushort_as_half(uint16_t(e.mlo))), fh = __half2float(__ushort_as_half(uint16_t(e.mhi)));
         sl = pack_bf16x2(fl, fl);
         sh = pack_bf16x2(fh, fh);
-        const uint32_t zbl = 0x4300u | (e.mlo >> 16), zbh = 0x4300u | (e.mhi >> 16);  // bf16(128 + z)
+        const int zsh = 4 * (((j * kMmaStepK + 32 * c) >> a.log2g) & 7);  // this step's group in its zero word
+        const uint32_t zbl = 0x4300u | ((e.zlo >> zsh) & 0xFu), zbh = 0x4300u | ((e.zhi >> zsh) & 0xFu);  // bf16(128 + z)
         zl2 = zbl | (zbl << 16);
         zh2 = zbh | (zbh << 16);
       } else {
