@@ -112,8 +112,10 @@ def test_split_k_plan_is_host_logic():
     # workspace query is the partial tiles' size (whole fp32 tiles, one wave of CTAs at
     # most) and 0 when nothing splits
     split = [(512, 256, 11008), (512, 2048, 11008), (2048, 256, 4096), (512, 256, 2048), (512, 2048, 2048),
-             (2048, 2048, 11008)]
-    unsplit = [(8192, 11008, 2048), (2048, 2048, 2048), (16, 256, 11008), (512, 11008, 2048)]
+             (2048, 2048, 11008), (512, 2560, 2048)]
+    # (the last three: q/k/v and gate/up stacked along N, whose tiles fill the SMs)
+    unsplit = [(8192, 11008, 2048), (2048, 2048, 2048), (16, 256, 11008), (512, 11008, 2048),
+               (2048, 2560, 2048), (2048, 22016, 2048), (8192, 2560, 2048)]
     for M, N, K in split:
         for fmt in (wq.WQ_FMT_INT4, wq.WQ_FMT_NVFP4):
             ws = wq.linear_workspace_size(M, N, K, fmt)
